@@ -1,0 +1,194 @@
+/*
+ * awq_w4a16.h -- C ABI of a W4A16 group-quantized linear layer (AWQ) for NVIDIA B200 (sm_100a).
+ *
+ * The layer computes  y = x' . dequant(W)^T  where W is an N x K (out x in) weight quantized to unsigned
+ * 4-bit codes with one fp16 scale and one 4-bit zero point per group of 128 consecutive input channels,
+ * dequantized as (q - z) * scale, and x' is the fp16 activation with the AWQ per-input-channel scale
+ * divided out.  Sources (web pages on AWQ; each cited by title and section):
+ *   [AWQ/GPTQ]   "AWQ and GPTQ algorithms" (jsqmd.com), section 2.1 (2) importance E[|X_j|],
+ *                section 2.1 (3) channel scaling: multiply salient weight channels by s, divide the
+ *                activations by s at inference, mathematically equivalent before rounding;
+ *                section 1.1: W4A16 = 4-bit weights, fp16 activations.
+ *   [LLM-AWQ]    "LLM-AWQ academic impact" (blog.csdn.net mirror), section "quantization flow":
+ *                --w_bit 4 --q_group_size 128, two stages (scale search, then real quantization).
+ *   [AutoAWQ]    "LLM quantization speed-up" (bjdmk.com.cn), section "quantization parameters":
+ *                group size 128, zero-point quantization, GEMV mode (single batch) vs GEMM mode.
+ * Where the pages leave a step open, the library takes the plain reading stated at each entry point.
+ *
+ * Conventions (all entry points):
+ *   - Pointers named d_* are DEVICE pointers (global memory of the current CUDA device).  The caller
+ *     allocates and frees every buffer; the library never allocates device memory and never
+ *     synchronizes, except awq_last_device_status().
+ *   - fp16 values are passed as uint16_t bit patterns (IEEE binary16).
+ *   - Every call enqueues its kernels on `stream` (a cudaStream_t; NULL = legacy default stream) and
+ *     returns at once.  Arguments are checked on the host first; on failure the call returns the
+ *     status code and launches nothing.  A launch failure returns AWQ_ERR_CUDA.
+ *   - Device pointers must be 16-byte aligned (AWQ_ERR_MISALIGNED otherwise).
+ *   - NaN or Inf anywhere in W, s, xcal or x is undefined behaviour (not checked).
+ *   - Kernels launched by this library call griddepcontrol.wait before they read any activation or
+ *     write any output, so they may be launched with programmatic dependent launch; they read only
+ *     packed weights before that point.
+ *
+ * ---------------------------------------------------------------------------------------------------
+ * PACKED WEIGHT LAYOUT (this library's own; the producer is awq_pack)
+ *
+ *   N_pad = N rounded up to a multiple of 32.   G = K / 128.   Row n, input channel k.
+ *
+ *   qweight  uint32_t[N_pad * K / 8].  The rows are cut into row blocks of 32 rows (rb = n / 32,
+ *            r = n % 32) and K into chunks of 32 channels (kc = k / 32).  Each (rb, kc) tile is 512
+ *            contiguous bytes: 32 rows x 4 words, row r's 4 words at word offset 4*r.  Tiles are stored
+ *            row-block major:  tile (rb, kc) begins at word  (rb * (K/32) + kc) * 128.
+ *            Word j (0..3) of row r in tile (rb, kc) holds the 8 codes of channels
+ *            k = 32*kc + 8*j + e, e = 0..7, in nibbles (bits 4p..4p+3, p = 0..7) ordered so that
+ *              nibble p = e/2      holds the code of even e,
+ *              nibble p = 4 + e/2  holds the code of odd e;
+ *            i.e. nibble order e = [0, 2, 4, 6, 1, 3, 5, 7].  (Masking the word with 0x000F000F puts
+ *            channels e=0,1 in the two 16-bit halves; 0x00F000F0 gives e=2,3; the word shifted right by
+ *            8 gives e=4,5 and e=6,7 the same way.)
+ *            Consequence: the 32 rows x 128 channels of one (row block, group) are 2048 contiguous
+ *            bytes starting at byte (rb * G + g) * 2048.
+ *   scales   uint16_t (fp16)[G * N_pad], group major: the scale of row n, group g is scales[g*N_pad + n].
+ *   qzeros   uint32_t[G * N_pad / 8], group major: the zero of row n, group g is nibble (n % 8)
+ *            (bits 4*(n%8) .. +3) of word qzeros[g*(N_pad/8) + n/8].
+ *   Padding rows n = N .. N_pad-1 hold code 0, scale 0 and zero 0 in every array.
+ *   Bytes per weight (N a multiple of 32): 0.5 + 2/128 + 0.5/128 = 0.51953.
+ *
+ * QUANTIZATION GRID (what awq_pack computes; plain reading of [AutoAWQ] zero point + [LLM-AWQ] w_bit 4,
+ * q_group_size 128 as asymmetric min/max round-to-nearest), per row n and group g, all in IEEE fp32
+ * with correctly rounded operations and no fused multiply-add:
+ *   w'_k  = W_nk * s_k                                   (exact: an fp16 x fp16 product fits fp32)
+ *   mn    = min_k w'_k,  mx = max_k w'_k                 (over the 128 channels of the group)
+ *   sc32  = max((mx - mn) / 15, 1e-5f);   sc = fp16_rne(sc32);   S = float(sc)
+ *   z     = clamp(rint(-mn / S), 0, 15)                  (rint = round half to even)
+ *   q_k   = clamp(rint(w'_k / S) + z, 0, 15)
+ * Dequantized weight: (q_k - z) * S.
+ * ---------------------------------------------------------------------------------------------------
+ */
+#ifndef AWQ_W4A16_H
+#define AWQ_W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum awq_status {
+  AWQ_OK = 0,
+  AWQ_ERR_INVALID_ARG = 1,     /* a size or pointer argument is out of range or NULL */
+  AWQ_ERR_UNSUPPORTED = 2,     /* a valid request this library does not implement (e.g. g != 128) */
+  AWQ_ERR_MISALIGNED = 3,      /* a device pointer is not 16-byte aligned */
+  AWQ_ERR_CUDA = 4,            /* a CUDA runtime call or kernel launch failed */
+  AWQ_ERR_DEVICE_TIMEOUT = 5,  /* a kernel gave up on a bounded wait (read via awq_last_device_status) */
+  AWQ_ERR_WORKSPACE = 6        /* the workspace is NULL or smaller than w4a16_workspace_bytes() */
+} awq_status;
+
+/* Opaque stream handle, ABI-compatible with cudaStream_t. */
+typedef struct CUstream_st* awq_stream_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* awq_status_string(awq_status st);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int awq_version(void);
+
+/*
+ * awq_packed_sizes -- byte sizes of the three packed arrays for an N x K weight at group size g
+ * (layout above).  Host only; launches nothing.
+ * Errors: AWQ_ERR_INVALID_ARG if N < 1, K < 1, K % g != 0 or an output pointer is NULL;
+ *         AWQ_ERR_UNSUPPORTED if g != 128.
+ */
+awq_status awq_packed_sizes(int N, int K, int g, size_t* qweight_bytes, size_t* scales_bytes,
+                            size_t* qzeros_bytes);
+
+/*
+ * awq_act_scale -- per-input-channel AWQ scale from calibration activations.
+ * [AWQ/GPTQ] section 2.1 (2): the statistic is the mean absolute activation E[|X_j|] over the
+ * calibration rows; the scale is that statistic raised to the exponent alpha = 0.5 (this library's fixed
+ * exponent; the scale search over alpha is not part of this entry point):
+ *     s_j = fp16_rne( sqrt( (sum_r |xcal_rj|) / R ) ),   sum, division and sqrt in IEEE fp64.
+ * (The fp64 sum of up to 8192 fp16 magnitudes is exact, so the result does not depend on order.)
+ *   d_xcal  [R][K] fp16, row major, device.        d_s  [K] fp16, device, written.
+ * Errors: AWQ_ERR_INVALID_ARG if R < 1, R > 8192, K < 1, or a pointer is NULL.
+ */
+awq_status awq_act_scale(const uint16_t* d_xcal, int R, int K, uint16_t* d_s, awq_stream_t stream);
+
+/*
+ * awq_apply_inv_scale -- divide the activations by the AWQ scale ([AWQ/GPTQ] section 2.1 (3):
+ * "activations are inverse-scaled at inference" so that x' . (W diag(s))^T = x . W^T before rounding):
+ *     x'_mk = fp16_rne( x_mk / s_k ),   the division in IEEE fp64.
+ *   d_x [M][K] fp16, d_s [K] fp16, d_xp [M][K] fp16 written (may alias d_x).  Device pointers.
+ * Errors: AWQ_ERR_INVALID_ARG if M < 1, K < 1, or a pointer is NULL.
+ */
+awq_status awq_apply_inv_scale(const uint16_t* d_x, const uint16_t* d_s, int M, int K, uint16_t* d_xp,
+                               awq_stream_t stream);
+
+/*
+ * awq_pack -- fold the AWQ scale into W, quantize with the grid above and write the packed layout.
+ * Bit-exact: the three arrays depend only on W, s, N, K.
+ *   d_W       [N][K] fp16, row major, device.
+ *   d_s       [K] fp16 per-input-channel scale, device; NULL means s = 1 (plain round-to-nearest).
+ *   d_qweight, d_scales, d_qzeros: outputs of awq_packed_sizes() bytes each (padding rows written).
+ * Errors: AWQ_ERR_INVALID_ARG (N < 1, K < 1, K % g != 0, NULL output), AWQ_ERR_UNSUPPORTED (g != 128),
+ *         AWQ_ERR_MISALIGNED, AWQ_ERR_CUDA.
+ */
+awq_status awq_pack(const uint16_t* d_W, const uint16_t* d_s, int N, int K, int g, uint32_t* d_qweight,
+                    uint16_t* d_scales, uint32_t* d_qzeros, awq_stream_t stream);
+
+/*
+ * The three linear-layer entry points share one argument list:
+ *   d_x       [M][K] fp16 activations (already divided by s), row major, device.
+ *   d_qweight, d_scales, d_qzeros: packed weight from awq_pack for the same N, K, g.
+ *   d_y       [M][N] fp16 output, row major, device; y_mn = fp16_rne(sum_k x'_mk (q_nk - z) S),
+ *             accumulated in fp32 (summation order is implementation defined).
+ *   M >= 1, N >= 1 with N % 8 == 0, K >= 128 with K % 128 == 0, g == 128.
+ *   d_workspace / workspace_bytes: device scratch of at least w4a16_workspace_bytes(mode, M, N, K, g)
+ *             bytes (may be NULL when that is 0).  The workspace must be zero-filled once before its
+ *             first use (cudaMemsetAsync); every call leaves it ready for the next call.  Calls that
+ *             share a workspace must not run concurrently on the GPU.
+ * Errors: AWQ_ERR_INVALID_ARG, AWQ_ERR_UNSUPPORTED, AWQ_ERR_MISALIGNED, AWQ_ERR_WORKSPACE, AWQ_ERR_CUDA.
+ */
+
+/* w4a16_gemv -- decode path ([AutoAWQ] "GEMV mode", single batch): CUDA-core kernel that streams the
+ * packed weights once per 8 rows of x with 128-bit loads, dequantizes in registers and accumulates
+ * in fp32; the input channels are split across warps and the partial sums are combined in the
+ * workspace.  Any M is accepted (M > 8 runs ceil(M/8) passes). */
+awq_status w4a16_gemv(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                      const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
+                      void* d_workspace, size_t workspace_bytes, awq_stream_t stream);
+
+/* w4a16_gemm -- prefill path ([AutoAWQ] "GEMM mode", long context): packed tiles staged by the TMA,
+ * dequantized to fp16 in shared memory and contracted on the 5th-generation tensor cores (tcgen05,
+ * fp32 accumulators in tensor memory). */
+awq_status w4a16_gemm(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                      const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
+                      void* d_workspace, size_t workspace_bytes, awq_stream_t stream);
+
+/* w4a16_linear -- picks GEMV when M <= w4a16_gemv_max_m(N, K), GEMM otherwise, and calls it. */
+awq_status w4a16_linear(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                        const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
+                        void* d_workspace, size_t workspace_bytes, awq_stream_t stream);
+
+/* Mode selector used by w4a16_linear: the largest M for which GEMV mode is chosen. */
+int w4a16_gemv_max_m(int N, int K);
+
+/* Modes for w4a16_workspace_bytes. */
+#define AWQ_MODE_GEMV 1
+#define AWQ_MODE_GEMM 2
+#define AWQ_MODE_LINEAR 3
+
+/* Workspace bytes a call needs on the current device (0 if none); SIZE_MAX for invalid sizes. */
+size_t w4a16_workspace_bytes(int mode, int M, int N, int K, int g);
+
+/*
+ * awq_last_device_status -- synchronizes `stream`, then reads and clears the device status word that
+ * kernels set when a bounded wait runs out.  Returns AWQ_OK, AWQ_ERR_DEVICE_TIMEOUT or AWQ_ERR_CUDA.
+ */
+awq_status awq_last_device_status(awq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AWQ_W4A16_H */

@@ -1,0 +1,256 @@
+/*
+ * awq_oracle.c -- CPU ORACLE for the W4A16 AWQ linear layer.  TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, single-threaded, slow and obviously correct.  It shares no code with the CUDA library: the
+ * fp16 conversions, the quantizer, the packed layout and the matmul are written here from the IEEE 754
+ * definitions, from the pages and from the prose layout description in the library's public header.
+ * Only the test suite, the smoke check and the CPU-baseline leg of the benchmark may load it.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC (x86-64 SSE2 arithmetic, so
+ * every float / double operation below is one correctly rounded IEEE operation).
+ *
+ * Sources (web pages on AWQ, cited by title and section):
+ *   [AWQ/GPTQ]  "AWQ and GPTQ algorithms" (jsqmd.com): section 2.1 (2) importance E[|X_j|] over the
+ *               calibration data; section 2.1 (3) multiply salient weight channels by s and divide the
+ *               activations by s at inference (equivalent before rounding); section 1.1 W4A16.
+ *   [LLM-AWQ]   "LLM-AWQ academic impact" (CSDN mirror), "quantization flow": w_bit 4, group size 128.
+ *   [AutoAWQ]   "LLM quantization speed-up" (bjdmk.com.cn), "quantization parameters": group 128,
+ *               zero-point quantization.
+ * Readings where the pages are silent (the same ones the public header states):
+ *   - grid: asymmetric min/max round-to-nearest over each group of 128 channels of one output row:
+ *     scale = max((max - min)/15, 1e-5) rounded to fp16, zero = clamp(rint(-min/scale), 0, 15),
+ *     q = clamp(rint(w/scale) + zero, 0, 15); fp32 arithmetic, rint = half to even;
+ *   - the AWQ scale exponent is 0.5: s = fp16((mean_r |x_rj|)^0.5), computed in fp64;
+ *   - activations: x' = fp16(x / s) with the division in fp64.
+ *
+ * Parity pins (each function is checked by tests/test_oracle_pins.py against something other than
+ * itself): numpy's float16 conversions, closed forms of the grid, the round-trip bound, q = z gives 0,
+ * s = 1 equals plain RTN, an independent unpacker, neutrality of the scaling in fp64, and brute-force
+ * matmuls.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------------------------------ */
+/* IEEE binary16 conversions, from the definition of the format (1 sign, 5 exponent, 10 fraction bits,
+ * bias 15, subnormals k * 2^-24).                                                                   */
+
+/* Exact widening of a binary16 bit pattern to double. */
+double oracle_f16_to_f64(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1F;
+  int f = h & 0x3FF;
+  double v;
+  if (e == 0x1F) {
+    v = f ? NAN : INFINITY;
+  } else if (e == 0) {
+    v = ldexp((double)f, -24); /* subnormal: f * 2^-24 */
+  } else {
+    v = ldexp((double)(1024 + f), e - 25); /* (1 + f/1024) * 2^(e-15) */
+  }
+  return sign ? -v : v;
+}
+
+float oracle_f16_to_f32(uint16_t h) { return (float)oracle_f16_to_f64(h); }
+
+/* Round a double to the nearest binary16, ties to even, in ONE rounding step. */
+uint16_t oracle_f64_to_f16(double d) {
+  uint64_t b;
+  memcpy(&b, &d, sizeof b);
+  uint16_t sign = (uint16_t)((b >> 63) << 15);
+  int e = (int)((b >> 52) & 0x7FF);
+  uint64_t m = b & ((1ULL << 52) - 1);
+  if (e == 0x7FF) return (uint16_t)(sign | 0x7C00 | (m ? 0x200 : 0)); /* Inf or (quiet) NaN */
+  if (e == 0) return sign;            /* zero or a double subnormal: far below half of 2^-24 */
+  int E = e - 1023;                   /* value = S * 2^(E - 52), S = 2^52 + m */
+  if (E > 15) return (uint16_t)(sign | 0x7C00);
+  uint64_t S = (1ULL << 52) | m;
+  int qexp = (E > -14 ? E : -14) - 10; /* exponent of one unit in the last place of the result */
+  int r = 52 + qexp - E;              /* bits of S below that unit */
+  if (r >= 54) return sign;           /* value < half the smallest subnormal */
+  uint64_t k = S >> r;
+  uint64_t rem = S & ((1ULL << r) - 1);
+  uint64_t half = 1ULL << (r - 1);
+  if (rem > half || (rem == half && (k & 1))) k += 1;
+  uint32_t out;
+  if (E >= -14) {
+    out = ((uint32_t)(E + 14) << 10) + (uint32_t)k; /* k in [1024, 2048]; 2048 carries into exponent */
+  } else {
+    out = (uint32_t)k; /* subnormal; k == 1024 is exactly the smallest normal */
+  }
+  if (out >= 0x7C00) return (uint16_t)(sign | 0x7C00);
+  return (uint16_t)(sign | out);
+}
+
+/* float -> binary16: widening to double is exact, so this is one rounding of the float's value. */
+uint16_t oracle_f32_to_f16(float f) { return oracle_f64_to_f16((double)f); }
+
+/* ------------------------------------------------------------------------------------------------ */
+/* Step a1: per-channel AWQ scale ([AWQ/GPTQ] 2.1 (2), exponent 0.5).                               */
+void oracle_act_scale(const uint16_t* xcal, int R, int K, uint16_t* s) {
+  for (int j = 0; j < K; ++j) {
+    double sum = 0.0;
+    for (int r = 0; r < R; ++r) sum += fabs(oracle_f16_to_f64(xcal[(size_t)r * K + j]));
+    double mean = sum / (double)R;
+    s[j] = oracle_f64_to_f16(sqrt(mean));
+  }
+}
+
+/* Step a7: activations divided by s ([AWQ/GPTQ] 2.1 (3)). */
+void oracle_inv_scale(const uint16_t* x, const uint16_t* s, int M, int K, uint16_t* xp) {
+  for (int m = 0; m < M; ++m)
+    for (int k = 0; k < K; ++k) {
+      size_t i = (size_t)m * K + k;
+      xp[i] = oracle_f64_to_f16(oracle_f16_to_f64(x[i]) / oracle_f16_to_f64(s[k]));
+    }
+}
+
+/* ------------------------------------------------------------------------------------------------ */
+/* Steps a2-a5: fold s into W and quantize each (row, group) with the asymmetric 4-bit grid.
+ *   W [N][K] fp16, s [K] fp16 or NULL (= 1).  Outputs, unpacked: q [N][K] codes 0..15,
+ *   sc [N][K/g] fp16 scales, z [N][K/g] zeros 0..15.                                                 */
+void oracle_quantize(const uint16_t* W, const uint16_t* s, int N, int K, int g, uint8_t* q, uint16_t* sc,
+                     uint8_t* z) {
+  int G = K / g;
+  float* wp = (float*)malloc(sizeof(float) * (size_t)g);
+  for (int n = 0; n < N; ++n) {
+    for (int gi = 0; gi < G; ++gi) {
+      /* a2: w' = W * s in fp32 (exact) */
+      for (int e = 0; e < g; ++e) {
+        int k = gi * g + e;
+        float w = oracle_f16_to_f32(W[(size_t)n * K + k]);
+        float sk = s ? oracle_f16_to_f32(s[k]) : 1.0f;
+        wp[e] = w * sk;
+      }
+      /* a3: group min and max */
+      float mn = wp[0], mx = wp[0];
+      for (int e = 1; e < g; ++e) {
+        if (wp[e] < mn) mn = wp[e];
+        if (wp[e] > mx) mx = wp[e];
+      }
+      /* a4: scale (fp16) and zero point */
+      float range = mx - mn;
+      float sc32 = range / 15.0f;
+      if (sc32 < 1e-5f) sc32 = 1e-5f;
+      uint16_t sch = oracle_f32_to_f16(sc32);
+      float S = oracle_f16_to_f32(sch);
+      float zf = rintf(-mn / S);
+      if (zf < 0.0f) zf = 0.0f;
+      if (zf > 15.0f) zf = 15.0f;
+      int zi = (int)zf;
+      sc[(size_t)n * G + gi] = sch;
+      z[(size_t)n * G + gi] = (uint8_t)zi;
+      /* a5: codes */
+      for (int e = 0; e < g; ++e) {
+        float r = rintf(wp[e] / S);
+        float v = r + (float)zi;
+        if (v < 0.0f) v = 0.0f;
+        if (v > 15.0f) v = 15.0f;
+        q[(size_t)n * K + gi * g + e] = (uint8_t)(int)v;
+      }
+    }
+  }
+  free(wp);
+}
+
+/* ------------------------------------------------------------------------------------------------ */
+/* Step a6: write the packed layout described in the public header (prose), from unpacked q, sc, z.
+ * Rows N .. N_pad-1 are zero.                                                                       */
+static int round_up32(int n) { return (n + 31) / 32 * 32; }
+
+void oracle_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int N, int K, int g,
+                 uint32_t* qweight, uint16_t* scales, uint32_t* qzeros) {
+  int G = K / g;
+  int Np = round_up32(N);
+  int KC = K / 32;
+  memset(qweight, 0, sizeof(uint32_t) * (size_t)Np * K / 8);
+  memset(scales, 0, sizeof(uint16_t) * (size_t)G * Np);
+  memset(qzeros, 0, sizeof(uint32_t) * (size_t)G * Np / 8);
+  /* nibble position of channel offset e inside a word: even e -> e/2, odd e -> 4 + e/2 */
+  for (int n = 0; n < N; ++n) {
+    int rb = n / 32, r = n % 32;
+    for (int k = 0; k < K; ++k) {
+      int kc = k / 32, j = (k % 32) / 8, e = k % 8;
+      int p = (e % 2 == 0) ? e / 2 : 4 + e / 2;
+      size_t word = ((size_t)rb * KC + kc) * 128 + (size_t)r * 4 + j;
+      qweight[word] |= (uint32_t)(q[(size_t)n * K + k] & 0xF) << (4 * p);
+    }
+    for (int gi = 0; gi < G; ++gi) {
+      scales[(size_t)gi * Np + n] = sc[(size_t)n * G + gi];
+      qzeros[(size_t)gi * (Np / 8) + n / 8] |= (uint32_t)(z[(size_t)n * G + gi] & 0xF) << (4 * (n % 8));
+    }
+  }
+}
+
+/* Independent decoder of the packed layout (used to pin oracle_pack by round trip).  It walks the
+ * packed words in storage order and asks, for every nibble, which (row, channel) it belongs to. */
+void oracle_unpack(const uint32_t* qweight, const uint16_t* scales, const uint32_t* qzeros, int N, int K,
+                   int g, uint8_t* q, uint16_t* sc, uint8_t* z) {
+  int G = K / g;
+  int Np = round_up32(N);
+  size_t nwords = (size_t)Np * K / 8;
+  static const int chan_of_nibble[8] = {0, 2, 4, 6, 1, 3, 5, 7};
+  for (size_t w = 0; w < nwords; ++w) {
+    size_t tile = w / 128;            /* 512-byte tile index = rb * (K/32) + kc */
+    int within = (int)(w % 128);      /* 32 rows x 4 words */
+    int r = within / 4, j = within % 4;
+    int rb = (int)(tile / (size_t)(K / 32)), kc = (int)(tile % (size_t)(K / 32));
+    int n = rb * 32 + r;
+    for (int p = 0; p < 8; ++p) {
+      int k = kc * 32 + j * 8 + chan_of_nibble[p];
+      uint8_t code = (uint8_t)((qweight[w] >> (4 * p)) & 0xF);
+      if (n < N) q[(size_t)n * K + k] = code;
+    }
+  }
+  for (int gi = 0; gi < G; ++gi)
+    for (int n = 0; n < N; ++n) {
+      sc[(size_t)n * G + gi] = scales[(size_t)gi * Np + n];
+      z[(size_t)n * G + gi] = (uint8_t)((qzeros[(size_t)gi * (Np / 8) + n / 8] >> (4 * (n % 8))) & 0xF);
+    }
+}
+
+/* ------------------------------------------------------------------------------------------------ */
+/* Exact dequantization: Wq = (q - z) * S in fp32 (|q - z| <= 15 times an 11-bit significand: exact). */
+void oracle_dequant(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int N, int K, int g, float* Wq) {
+  int G = K / g;
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) {
+      int gi = k / g;
+      float S = oracle_f16_to_f32(sc[(size_t)n * G + gi]);
+      int d = (int)q[(size_t)n * K + k] - (int)z[(size_t)n * G + gi];
+      Wq[(size_t)n * K + k] = (float)d * S;
+    }
+}
+
+/* y[m][n] = sum_k x'[m][k] * Wq[n][k], plain triple loop accumulated in fp64. */
+void oracle_linear_f64(const uint16_t* xp, const float* Wq, int M, int N, int K, double* y) {
+  for (int m = 0; m < M; ++m)
+    for (int n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int k = 0; k < K; ++k)
+        acc += oracle_f16_to_f64(xp[(size_t)m * K + k]) * (double)Wq[(size_t)n * K + k];
+      y[(size_t)m * N + n] = acc;
+    }
+}
+
+/* Sampled outputs straight from the unpacked quantization: y for the listed (m, n) pairs, fp64. */
+void oracle_linear_pairs_f64(const uint16_t* xp, const uint8_t* q, const uint16_t* sc, const uint8_t* z,
+                             int M, int N, int K, int g, const int32_t* ms, const int32_t* ns, int count,
+                             double* out) {
+  int G = K / g;
+  (void)M;
+  (void)N;
+  for (int i = 0; i < count; ++i) {
+    int m = ms[i], n = ns[i];
+    double acc = 0.0;
+    for (int k = 0; k < K; ++k) {
+      int gi = k / g;
+      double S = oracle_f16_to_f64(sc[(size_t)n * G + gi]);
+      int d = (int)q[(size_t)n * K + k] - (int)z[(size_t)n * G + gi];
+      acc += oracle_f16_to_f64(xp[(size_t)m * K + k]) * ((double)d * S);
+    }
+    out[i] = acc;
+  }
+}

@@ -1,0 +1,201 @@
+"""CPU oracle for the W4A16 AWQ linear layer -- TEST INFRASTRUCTURE ONLY.
+
+Thin ctypes wrapper around ``awq_oracle.c`` (plain single-threaded C, fp32 quantizer and fp64 matmul).
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import this
+module.  It shares no code with the CUDA library under ``weight_only_int4_05_b200/``.
+
+Every function states the step of the method it follows; the pins that tie it to something other than
+itself live in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "awq_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+GROUP = 128
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE arithmetic: no fast-math, no FMA contraction)."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".{os.getpid()}.tmp"
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+               _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            lib.oracle_f16_to_f64.restype = ctypes.c_double
+            lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
+            lib.oracle_f64_to_f16.restype = ctypes.c_uint16
+            lib.oracle_f64_to_f16.argtypes = [ctypes.c_double]
+            lib.oracle_f32_to_f16.restype = ctypes.c_uint16
+            lib.oracle_f32_to_f16.argtypes = [ctypes.c_float]
+            lib.oracle_act_scale.argtypes = [P, I, I, P]
+            lib.oracle_inv_scale.argtypes = [P, P, I, I, P]
+            lib.oracle_quantize.argtypes = [P, P, I, I, I, P, P, P]
+            lib.oracle_pack.argtypes = [P, P, P, I, I, I, P, P, P]
+            lib.oracle_unpack.argtypes = [P, P, P, I, I, I, P, P, P]
+            lib.oracle_dequant.argtypes = [P, P, P, I, I, I, P]
+            lib.oracle_linear_f64.argtypes = [P, P, I, I, I, P]
+            lib.oracle_linear_pairs_f64.argtypes = [P, P, P, P, I, I, I, I, P, P, I, P]
+            for name in ("oracle_act_scale", "oracle_inv_scale", "oracle_quantize", "oracle_pack",
+                         "oracle_unpack", "oracle_dequant", "oracle_linear_f64", "oracle_linear_pairs_f64"):
+                getattr(lib, name).restype = None
+            _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float16:
+        a = a.view(np.uint16)
+    assert a.dtype == np.uint16
+    return a
+
+
+# ---- fp16 conversions (IEEE binary16 from its definition) -----------------------------------------
+def f16_to_f64(h: int) -> float:
+    return _load().oracle_f16_to_f64(int(h))
+
+
+def f64_to_f16(d: float) -> int:
+    return int(_load().oracle_f64_to_f16(float(d)))
+
+
+def f32_to_f16(f: float) -> int:
+    return int(_load().oracle_f32_to_f16(float(np.float32(f))))
+
+
+# ---- a1: AWQ per-channel scale --------------------------------------------------------------------
+def act_scale(xcal) -> np.ndarray:
+    """s_j = fp16(sqrt(mean_r |xcal_rj|)) in fp64 ("AWQ and GPTQ algorithms", section 2.1 (2))."""
+    xcal = _u16(xcal)
+    R, K = xcal.shape
+    s = np.empty(K, np.uint16)
+    _load().oracle_act_scale(_p(xcal), R, K, _p(s))
+    return s
+
+
+# ---- a7: x' = x / s -------------------------------------------------------------------------------
+def inv_scale(x, s) -> np.ndarray:
+    """x'_mk = fp16(x_mk / s_k), fp64 division ("AWQ and GPTQ algorithms", section 2.1 (3))."""
+    x = _u16(x)
+    s = _u16(s)
+    M, K = x.shape
+    xp = np.empty_like(x)
+    _load().oracle_inv_scale(_p(x), _p(s), M, K, _p(xp))
+    return xp
+
+
+# ---- a2..a5: fold + grid + codes ------------------------------------------------------------------
+def quantize(W, s=None, g: int = GROUP):
+    """Returns (q [N][K] uint8, sc [N][G] uint16 fp16 bits, z [N][G] uint8)."""
+    W = _u16(W)
+    N, K = W.shape
+    G = K // g
+    q = np.empty((N, K), np.uint8)
+    sc = np.empty((N, G), np.uint16)
+    z = np.empty((N, G), np.uint8)
+    sp = None if s is None else _p(_u16(s))
+    _load().oracle_quantize(_p(W), sp, N, K, g, _p(q), _p(sc), _p(z))
+    return q, sc, z
+
+
+def packed_sizes(N: int, K: int, g: int = GROUP):
+    Np = (N + 31) // 32 * 32
+    G = K // g
+    return Np * K // 2, G * Np * 2, G * Np // 2
+
+
+# ---- a6: packed layout ----------------------------------------------------------------------------
+def pack(q, sc, z, g: int = GROUP):
+    N, K = q.shape
+    Np = (N + 31) // 32 * 32
+    G = K // g
+    qw = np.empty(Np * K // 8, np.uint32)
+    scales = np.empty(G * Np, np.uint16)
+    qz = np.empty(G * Np // 8, np.uint32)
+    _load().oracle_pack(_p(np.ascontiguousarray(q)), _p(np.ascontiguousarray(sc)),
+                        _p(np.ascontiguousarray(z)), N, K, g, _p(qw), _p(scales), _p(qz))
+    return qw, scales, qz
+
+
+def unpack(qw, scales, qz, N: int, K: int, g: int = GROUP):
+    G = K // g
+    q = np.empty((N, K), np.uint8)
+    sc = np.empty((N, G), np.uint16)
+    z = np.empty((N, G), np.uint8)
+    _load().oracle_unpack(_p(np.ascontiguousarray(qw)), _p(np.ascontiguousarray(scales)),
+                          _p(np.ascontiguousarray(qz)), N, K, g, _p(q), _p(sc), _p(z))
+    return q, sc, z
+
+
+def awq_pack(W, s=None, g: int = GROUP):
+    """Stage-2 "real quantization": fold s, quantize and pack.  Returns (qweight, scales, qzeros)."""
+    return pack(*quantize(W, s, g), g)
+
+
+# ---- dequant and matmul ---------------------------------------------------------------------------
+def dequant(q, sc, z, g: int = GROUP) -> np.ndarray:
+    N, K = q.shape
+    Wq = np.empty((N, K), np.float32)
+    _load().oracle_dequant(_p(np.ascontiguousarray(q)), _p(np.ascontiguousarray(sc)),
+                           _p(np.ascontiguousarray(z)), N, K, g, _p(Wq))
+    return Wq
+
+
+def linear_f64(xp, Wq) -> np.ndarray:
+    """y = x' . Wq^T, plain triple loop in fp64."""
+    xp = _u16(xp)
+    Wq = np.ascontiguousarray(Wq, dtype=np.float32)
+    M, K = xp.shape
+    N = Wq.shape[0]
+    y = np.empty((M, N), np.float64)
+    _load().oracle_linear_f64(_p(xp), _p(Wq), M, N, K, _p(y))
+    return y
+
+
+def linear_pairs_f64(xp, q, sc, z, ms, ns, g: int = GROUP) -> np.ndarray:
+    """y[m, n] for the listed pairs only (sampled parity at full size)."""
+    xp = _u16(xp)
+    M, K = xp.shape
+    N = q.shape[0]
+    ms = np.ascontiguousarray(ms, dtype=np.int32)
+    ns = np.ascontiguousarray(ns, dtype=np.int32)
+    out = np.empty(len(ms), np.float64)
+    _load().oracle_linear_pairs_f64(_p(xp), _p(np.ascontiguousarray(q)), _p(np.ascontiguousarray(sc)),
+                                    _p(np.ascontiguousarray(z)), M, N, K, g, _p(ms), _p(ns), len(ms),
+                                    _p(out))
+    return out
+
+
+def reference_linear(xp, W, s=None, g: int = GROUP) -> np.ndarray:
+    """Whole path from fp16 W: quantize (with s folded) then the fp64 matmul against x'."""
+    q, sc, z = quantize(W, s, g)
+    return linear_f64(xp, dequant(q, sc, z, g))

@@ -1,0 +1,415 @@
+"""Pins of the CPU oracle against things other than itself (CPU only).
+
+Each test names the oracle function it pins and what it is pinned to: numpy's IEEE conversions, a
+closed form obtained by construction, an invariant of the grid, a brute-force search, or a library
+routine that the special case reduces to.  A plausible slip in the oracle (a dropped term, a wrong
+sign, a transposed index) fails at least one of them.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_figures.txt")
+
+
+def f16(a):
+    return np.asarray(a, np.float16).view(np.uint16)
+
+
+def h2f(bits):
+    return np.asarray(bits, np.uint16).view(np.float16).astype(np.float64)
+
+
+# ---------------------------------------------------------------- fp16 conversions ---------------
+def test_f16_widening_matches_numpy_all_patterns():
+    """oracle_f16_to_f64 vs numpy float16 -> float64 over all 65536 bit patterns."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([O.f16_to_f64(int(b)) for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def _narrowing_sample(rng):
+    # every fp16 value, every midpoint between neighbours (ties), and the midpoints nudged by
+    # 1 ulp of double either way, plus random doubles spanning subnormal .. overflow
+    h = np.arange(0, 0x7C00, dtype=np.uint16)
+    v = h.view(np.float16).astype(np.float64)
+    mids = (v[:-1] + v[1:]) / 2
+    nudged = np.concatenate([np.nextafter(mids, np.inf), np.nextafter(mids, -np.inf)])
+    rnd = np.exp(rng.uniform(np.log(1e-9), np.log(7e4), 200000))
+    vals = np.concatenate([v, mids, nudged, rnd, [65504.0, 65519.0, 65519.999, 65520.0, 1e9, 0.0]])
+    return np.concatenate([vals, -vals])
+
+
+def test_f64_to_f16_matches_numpy_single_rounding():
+    """oracle_f64_to_f16 vs numpy's direct float64 -> float16 (round to nearest even)."""
+    vals = _narrowing_sample(np.random.default_rng(1))
+    with np.errstate(over="ignore"):
+        ref = vals.astype(np.float16).view(np.uint16)
+    got = np.array([O.f64_to_f16(float(d)) for d in vals], np.uint16)
+    assert np.array_equal(got, ref)
+
+
+def test_f32_to_f16_matches_numpy():
+    """oracle_f32_to_f16 vs numpy float32 -> float16 on random float32 bit patterns and ties."""
+    rng = np.random.default_rng(2)
+    bits = rng.integers(0, 2**31, 300000, dtype=np.uint32)
+    bits = bits[(bits & 0x7F800000) != 0x7F800000]  # drop NaN / Inf patterns
+    vals = bits.view(np.float32)
+    vals = np.concatenate([vals, -vals, (h2f(np.arange(1, 0x7BFF)) + h2f(np.arange(2, 0x7C00))).astype(
+        np.float32) / np.float32(2)])
+    with np.errstate(over="ignore"):
+        ref = vals.astype(np.float16).view(np.uint16)
+    got = np.array([O.f32_to_f16(float(f)) for f in vals], np.uint16)
+    assert np.array_equal(got, ref)
+
+
+# ---------------------------------------------------------------- a1: AWQ scale ------------------
+def test_act_scale_closed_forms():
+    """oracle_act_scale: s_j = fp16(sqrt(mean_r |x_rj|)).  Columns built so that the mean absolute
+    value is a known perfect square: the sign pattern, the row count and the column index all matter."""
+    R, K = 64, 6
+    x = np.zeros((R, K), np.float64)
+    x[:, 0] = 4.0                                    # mean 4 -> 2
+    x[:, 1] = np.where(np.arange(R) % 2, 9.0, -9.0)  # |.| drops the sign: mean 9 -> 3
+    x[:, 2] = np.where(np.arange(R) < 16, 1.0, 0.0)  # mean 16/64 = 0.25 -> 0.5
+    x[:, 3] = -0.0625                                # mean 1/16 -> 0.25
+    x[:32, 4] = 2.0                                  # mean 1 -> 1
+    x[:, 5] = np.where(np.arange(R) % 4 == 0, -64.0, 0.0)  # mean 16 -> 4
+    s = O.act_scale(f16(x))
+    assert list(h2f(s)) == [2.0, 3.0, 0.5, 0.25, 1.0, 4.0]
+
+
+def test_act_scale_non_power_of_two_rows_matches_exact_rational():
+    """R = 3: mean = sum/3 is inexact; the result equals fp16 of the correctly rounded sqrt of the
+    correctly rounded fp64 quotient, computed here with exact rationals and math.sqrt."""
+    x = f16(np.array([[1.0, 0.5, 7.0], [2.0, -0.25, 1.0], [-4.0, 0.125, 0.0]]))
+    s = O.act_scale(x)
+    for j in range(3):
+        total = sum(Fraction(abs(v)) for v in h2f(x[:, j]))   # exact
+        mean = float(total / 3)                               # one rounding (Fraction -> float)
+        exp = np.array([math.sqrt(mean)]).astype(np.float16).view(np.uint16)[0]
+        assert s[j] == exp
+
+
+# ---------------------------------------------------------------- a7: x / s ----------------------
+def test_inv_scale_powers_of_two_exact():
+    """oracle_inv_scale: with s_k a power of two, x / s is exact in fp16; a multiply instead of a divide,
+    or indexing s by row, fails."""
+    rng = np.random.default_rng(3)
+    M, K = 3, 8
+    x = f16(rng.standard_normal((M, K)))
+    e = np.array([-2, -1, 0, 1, 2, 3, -3, 0])
+    s = f16(2.0 ** e)
+    xp = O.inv_scale(x, s)
+    assert np.array_equal(h2f(xp), h2f(x) / 2.0 ** e[None, :])
+
+
+def test_inv_scale_x_equal_s_gives_one():
+    s = f16(np.array([0.3, 1.7, 12.5, 0.001]))
+    x = np.stack([s, s])
+    assert np.all(h2f(O.inv_scale(x, s)) == 1.0)
+
+
+# ---------------------------------------------------------------- a2..a5: grid -------------------
+def _grid_group(S0, z0, codes):
+    return (np.asarray(codes, np.float64) - z0) * S0
+
+
+@pytest.mark.parametrize("S0,z0", [(0.0078125, 5), (0.13232421875, 8), (0.000244140625, 0),
+                                   (0.5, 15), (0.0029296875, 3)])
+def test_quantize_reproduces_its_own_grid(S0, z0):
+    """By construction: a group whose values are exactly (j - z0) * S0 for j covering 0..15 has
+    range 15 * S0, so the scale is S0, the zero is z0 and every code is recovered (closed form)."""
+    rng = np.random.default_rng(int(S0 * 1e6) + z0)
+    codes = np.concatenate([np.arange(16), rng.integers(0, 16, 128 - 16)])
+    rng.shuffle(codes)
+    w = _grid_group(S0, z0, codes)
+    W = f16(w[None, :])
+    assert np.array_equal(h2f(W)[0], w)  # the construction is exact in fp16
+    q, sc, z = O.quantize(W)
+    assert h2f(sc)[0, 0] == S0 and z[0, 0] == z0
+    assert np.array_equal(q[0], codes)
+    assert np.array_equal(O.dequant(q, sc, z)[0].astype(np.float64), w)
+
+
+def test_quantize_all_positive_group_clamps_zero_and_top():
+    """All values > 0: -min/S < 0 so the zero clamps to 0, and values above 15.5 S clamp to code 15."""
+    w = np.linspace(1.0, 2.0, 128)
+    q, sc, z = O.quantize(f16(w[None, :]))
+    S = h2f(sc)[0, 0]
+    assert z[0, 0] == 0
+    assert q[0].max() == 15 and np.all(q[0][h2f(f16(w)) > 15.5 * S] == 15)
+
+
+def test_quantize_degenerate_group():
+    """max == min: the scale takes its floor 1e-5 (fp16 of it) and no code leaves 0..15."""
+    for c in (0.0, 0.37, -0.37):
+        q, sc, z = O.quantize(f16(np.full((1, 128), c)))
+        assert sc[0, 0] == f16(np.float32(1e-5))[()]
+        assert 0 <= q.min() and q.max() <= 15 and 0 <= z[0, 0] <= 15
+        if c == 0.0:
+            assert np.all(q[0] == z[0, 0])  # zero maps to the zero point exactly
+
+
+def _synthetic_group_rows(N=16, K=512, seed=5):
+    d = synth.linear_inputs(seed, 0, 0, 0, 1, N, K)
+    s = O.act_scale(d["xcal"])
+    return d["W"].view(np.uint16), s
+
+
+def test_quantize_roundtrip_bound():
+    """Invariant: for groups with min <= 0 <= max, |w' - (q - z) S| <= S (1/2 + 16 * 2^-11) for every
+    element (1/2 from rounding to the grid; the rest from rounding the scale to fp16)."""
+    W, s = _synthetic_group_rows()
+    q, sc, z = O.quantize(W, s)
+    wp = h2f(W) * h2f(s)[None, :]           # exact fold in fp64
+    deq = O.dequant(q, sc, z).astype(np.float64)
+    S = np.repeat(h2f(sc), 128, axis=1)
+    assert np.all(np.abs(wp - deq) <= S * (0.5 + 16 * 2.0**-11))
+
+
+def test_quantize_codes_are_nearest_grid_points_brute_force():
+    """Brute force: given (S, z), each code is the nearest of the 16 grid points (j - z) S to w',
+    and z is the grid offset nearest to -min/S; ties within 1e-6 S are skipped."""
+    W, s = _synthetic_group_rows(N=8, K=256)
+    q, sc, z = O.quantize(W, s)
+    wp = h2f(W) * h2f(s)[None, :]
+    G = 2
+    for n in range(W.shape[0]):
+        for g in range(G):
+            S = h2f(sc)[n, g]
+            zz = int(z[n, g])
+            grp = wp[n, g * 128:(g + 1) * 128]
+            dz = np.abs(-grp.min() / S - np.arange(16))
+            if np.sort(dz)[1] - np.sort(dz)[0] > 1e-6:
+                assert zz == int(np.argmin(dz))
+            for e, v in enumerate(grp):
+                d = np.abs(v - (np.arange(16) - zz) * S)
+                srt = np.sort(d)
+                if srt[1] - srt[0] > 1e-6 * S:
+                    assert q[n, g * 128 + e] == int(np.argmin(d))
+
+
+def test_quantize_group_boundaries_are_per_row_and_per_group():
+    """Groups of 128 along K within each row: a row whose second group is 8x larger gets an 8x scale
+    there and nowhere else; a transposed or misaligned group index fails."""
+    base = np.tile(np.linspace(-0.5, 0.5, 128), 2)
+    W = np.stack([base, base * np.r_[np.ones(128), 8 * np.ones(128)], base * 0.25])
+    q, sc, z = O.quantize(f16(W))
+    S = h2f(sc)
+    assert S[1, 0] == S[0, 0] and S[1, 1] == 8 * S[0, 1] and S[2, 0] == S[0, 0] / 4
+    assert np.array_equal(q[0], q[1]) and np.array_equal(q[0], q[2])
+
+
+def test_quantize_fold_direction_with_power_of_two_scale():
+    """Fold a2: quantize(W, s) equals quantize(fp16(W * s), s = 1) when s is a power of two (the
+    product is then exact in fp16); dividing by s instead fails."""
+    rng = np.random.default_rng(7)
+    W = f16(0.02 * rng.standard_normal((4, 256)))
+    s = f16(2.0 ** rng.integers(-2, 3, 256))
+    a = O.quantize(W, s)
+    b = O.quantize(f16(h2f(W) * h2f(s)[None, :]))
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+
+
+def test_quantize_s_none_equals_s_one():
+    """s = NULL means s = 1 (plain round-to-nearest, the baseline AWQ is compared with)."""
+    W, _ = _synthetic_group_rows(N=8, K=256)
+    a = O.quantize(W, None)
+    b = O.quantize(W, f16(np.ones(256)))
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+
+
+# ---------------------------------------------------------------- a6: packed layout --------------
+def _expected_location(n, k, K):
+    """Word index and bit offset of (n, k) read off the public header's prose layout description."""
+    rb, r, kc = n // 32, n % 32, k // 32
+    j, e = (k % 32) // 8, k % 8
+    p = e // 2 if e % 2 == 0 else 4 + e // 2
+    return (rb * (K // 32) + kc) * 128 + r * 4 + j, 4 * p
+
+
+def test_pack_single_nibble_placement():
+    """oracle_pack: a single nonzero code lands exactly at the word and nibble the header describes."""
+    N, K = 40, 256
+    rng = np.random.default_rng(11)
+    for _ in range(60):
+        n, k, c = int(rng.integers(N)), int(rng.integers(K)), int(rng.integers(1, 16))
+        q = np.zeros((N, K), np.uint8)
+        q[n, k] = c
+        qw, _, _ = O.pack(q, np.zeros((N, 2), np.uint16), np.zeros((N, 2), np.uint8))
+        word, bit = _expected_location(n, k, K)
+        exp = np.zeros_like(qw)
+        exp[word] = c << bit
+        assert np.array_equal(qw, exp)
+
+
+def test_pack_scales_and_zeros_placement_and_padding():
+    N, K = 40, 384  # N_pad = 64, G = 3
+    G, Np = 3, 64
+    rng = np.random.default_rng(12)
+    q = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    sc = f16(rng.uniform(0.001, 0.01, (N, G)))
+    z = rng.integers(0, 16, (N, G)).astype(np.uint8)
+    qw, scales, qz = O.pack(q, sc, z)
+    assert (qw.nbytes, scales.nbytes, qz.nbytes) == O.packed_sizes(N, K)
+    for n in range(Np):
+        for g in range(G):
+            got_s = scales[g * Np + n]
+            got_z = (qz[g * (Np // 8) + n // 8] >> (4 * (n % 8))) & 0xF
+            if n < N:
+                assert got_s == sc[n, g] and got_z == z[n, g]
+            else:
+                assert got_s == 0 and got_z == 0
+    # padding rows hold code 0: their whole 16-byte row slot in every tile is zero
+    words = qw.reshape(Np // 32, K // 32, 32, 4)
+    assert np.all(words[1, :, N - 32:, :] == 0)
+
+
+def test_pack_mask_property_stated_in_header():
+    """The header promises: word & 0x000F000F puts channels e=0,1 in the two 16-bit halves, 0x00F000F0
+    e=2,3, and the word >> 8 gives e=4,5 and e=6,7 the same way."""
+    N, K = 32, 32
+    codes = np.random.default_rng(13).integers(0, 16, (N, K)).astype(np.uint8)
+    qw, _, _ = O.pack(codes, np.zeros((N, 1), np.uint16), np.zeros((N, 1), np.uint8))
+    for r in range(N):
+        for j in range(4):
+            w = int(qw[r * 4 + j])
+            c = codes[r, 8 * j:8 * j + 8]
+            lo = lambda v: (v & 0xFFFF)  # noqa: E731
+            hi = lambda v: (v >> 16)     # noqa: E731
+            assert (lo(w & 0x000F000F), hi(w & 0x000F000F)) == (c[0], c[1])
+            assert (lo(w & 0x00F000F0) >> 4, hi(w & 0x00F000F0) >> 4) == (c[2], c[3])
+            w8 = w >> 8
+            assert (lo(w8 & 0x000F000F), hi(w8 & 0x000F000F)) == (c[4], c[5])
+            assert (lo(w8 & 0x00F000F0) >> 4, hi(w8 & 0x00F000F0) >> 4) == (c[6], c[7])
+
+
+def test_pack_unpack_roundtrip_independent_decoder():
+    """oracle_unpack (walks the storage in order) inverts oracle_pack (walks the matrix in order)."""
+    rng = np.random.default_rng(14)
+    for N, K in [(8, 128), (40, 256), (96, 512)]:
+        G = K // 128
+        q = rng.integers(0, 16, (N, K)).astype(np.uint8)
+        sc = rng.integers(0, 0x7BFF, (N, G)).astype(np.uint16)
+        z = rng.integers(0, 16, (N, G)).astype(np.uint8)
+        out = O.unpack(*O.pack(q, sc, z), N, K)
+        for a, b in zip(out, (q, sc, z)):
+            assert np.array_equal(a, b)
+
+
+def test_packed_bytes_match_page_memory_reduction():
+    """The page's "75% less memory" for W4A16 (AWQ and GPTQ algorithms, section 2.3) against the
+    packed size: (0.5 + 2/128 + 0.5/128) / 2 bytes per weight = 0.2598, a 74.0% reduction."""
+    figs = {}
+    for line in open(GOLDEN):
+        if line.strip() and not line.startswith("#"):
+            kv = line.split(";")[0]
+            k, v = kv.split("=")
+            figs[k.strip()] = float(v)
+    assert figs["q_group_size"] == O.GROUP and figs["w_bit"] == 4
+    N, K = 4096, 4096
+    total = sum(O.packed_sizes(N, K))
+    ratio = total / (2.0 * N * K)
+    assert abs(ratio - (0.5 + 2.5 / 128) / 2) < 1e-12
+    assert abs((1 - ratio) * 100 - figs["memory_reduction_percent"]) < 1.5
+
+
+# ---------------------------------------------------------------- dequant + matmul ---------------
+def test_dequant_zero_point_is_exact_zero_and_product_exact():
+    rng = np.random.default_rng(15)
+    N, K = 8, 256
+    q = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    z = rng.integers(0, 16, (N, 2)).astype(np.uint8)
+    q[:, :128] = z[:, :1]  # first group: every code equals the zero point
+    sc = f16(rng.uniform(1e-4, 0.5, (N, 2)))
+    Wq = O.dequant(q, sc, z)
+    assert np.all(Wq[:, :128] == 0.0)
+    exact = (q.astype(np.float64) - np.repeat(z, 128, axis=1)) * np.repeat(h2f(sc), 128, axis=1)
+    assert np.array_equal(Wq.astype(np.float64), exact)
+
+
+def test_linear_f64_brute_force_and_library():
+    """oracle_linear_f64 vs math.fsum over explicit products (brute force) and vs torch's CPU fp64
+    matmul, on non-square shapes so that a transposed operand fails."""
+    import torch
+
+    rng = np.random.default_rng(16)
+    for M, N, K in [(1, 16, 128), (3, 5, 256), (4, 16, 512)]:
+        xp = f16(rng.standard_normal((M, K)))
+        Wq = (rng.integers(-8, 8, (N, K)) * 0.01).astype(np.float32)
+        y = O.linear_f64(xp, Wq)
+        X = h2f(xp)
+        for m in range(M):
+            for n in range(N):
+                exact = math.fsum(float(X[m, k]) * float(Wq[n, k]) for k in range(K))
+                assert abs(y[m, n] - exact) <= 1e-12 * max(1.0, abs(exact))
+        ref = (torch.from_numpy(X) @ torch.from_numpy(Wq.astype(np.float64)).T).numpy()
+        assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_linear_f64_integer_exact():
+    """Integer-valued operands: the fp64 sum is exact, so y equals the integer matmul bit for bit."""
+    rng = np.random.default_rng(17)
+    M, N, K = 2, 7, 384
+    xi = rng.integers(-50, 50, (M, K))
+    wi = rng.integers(-15, 16, (N, K))
+    y = O.linear_f64(f16(xi.astype(np.float64)), wi.astype(np.float32))
+    assert np.array_equal(y, (xi @ wi.T).astype(np.float64))
+
+
+def test_linear_pairs_matches_full():
+    W, s = _synthetic_group_rows(N=24, K=384)
+    xp = f16(np.random.default_rng(18).standard_normal((3, 384)))
+    q, sc, z = O.quantize(W, s)
+    full = O.linear_f64(xp, O.dequant(q, sc, z))
+    ms, ns = np.meshgrid(np.arange(3), np.arange(24), indexing="ij")
+    pairs = O.linear_pairs_f64(xp, q, sc, z, ms.ravel(), ns.ravel())
+    assert np.array_equal(pairs, full.ravel())
+
+
+# ---------------------------------------------------------------- whole path ---------------------
+def test_awq_scaling_is_neutral_before_rounding():
+    """AWQ and GPTQ algorithms, section 2.1 (3): scaling weight channels by s and the activations by
+    1/s leaves x W^T unchanged.  With s a power of two every rounding in the oracle is exact, so the
+    whole path (fold, 1/s, quantize, matmul) must equal the same path on fp16(W s) and x / s computed
+    here exactly; and in fp64 with arbitrary s the identity holds to 1e-12."""
+    rng = np.random.default_rng(19)
+    M, N, K = 2, 16, 256
+    W = f16(0.02 * rng.standard_normal((N, K)))
+    x = f16(rng.standard_normal((M, K)))
+    e = rng.integers(-3, 4, K)
+    s = f16(2.0 ** e)
+    y_awq = O.reference_linear(O.inv_scale(x, s), W, s)
+    y_ref = O.reference_linear(f16(h2f(x) / 2.0 ** e), f16(h2f(W) * 2.0 ** e))
+    assert np.array_equal(y_awq, y_ref)
+    sa = rng.uniform(0.3, 3.0, K)
+    Wd, xd = h2f(W), h2f(x)
+    a = (xd / sa) @ (Wd * sa).T
+    b = xd @ Wd.T
+    assert np.max(np.abs(a - b)) <= 1e-12 * np.max(np.abs(b))
+
+
+def test_quantized_linear_within_grid_error_bound():
+    """|y_q - x' (W s)^T| <= sum_k |x'_k| S_{g(k)} (1/2 + 16 * 2^-11): the layer's error is bounded by
+    the per-element grid bound (a dropped zero point or scale breaks it)."""
+    d = synth.linear_inputs(21, 0, 0, 0, 2, 32, 512)
+    s = O.act_scale(d["xcal"])
+    xp = O.inv_scale(d["x"], s)
+    q, sc, z = O.quantize(d["W"], s)
+    yq = O.linear_f64(xp, O.dequant(q, sc, z))
+    y = h2f(xp) @ (h2f(d["W"]) * h2f(s)[None, :]).T
+    S = np.repeat(h2f(sc), 128, axis=1)
+    bound = np.abs(h2f(xp)) @ (S * (0.5 + 16 * 2.0**-11)).T
+    assert np.all(np.abs(yq - y) <= bound)
