@@ -1,0 +1,100 @@
+"""C ABI checks that need no GPU: the library builds, loads, exports every symbol the public header
+declares, and rejects bad arguments on the host (no kernel is launched on these paths)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from weight_only_int4_05_b200 import _lib, build as libbuild
+from oracle import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "awq_w4a16.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    libbuild.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if not n.startswith("defined")))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for n in ("awq_pack", "w4a16_gemv", "w4a16_gemm", "w4a16_linear", "awq_act_scale", "awq_apply_inv_scale"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert set(declared_functions()) == set(_lib.EXPORTS)
+
+
+def test_version_and_status_strings(L):
+    assert L.awq_version() == 100
+    for code, name in _lib.STATUS_NAMES.items():
+        assert L.awq_status_string(code).decode() == name
+
+
+@pytest.mark.parametrize("N,K", [(256, 512), (40, 384), (14336, 4096), (8, 128), (28672, 8192)])
+def test_packed_sizes_match_layout(L, N, K):
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.awq_packed_sizes(N, K, 128, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)) == 0
+    assert (a.value, b.value, c.value) == O.packed_sizes(N, K)
+
+
+def test_packed_sizes_rejects(L):
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    ref = (ctypes.byref(a), ctypes.byref(b), ctypes.byref(c))
+    assert L.awq_packed_sizes(256, 512, 64, *ref) == 2      # g != 128: unsupported
+    assert L.awq_packed_sizes(0, 512, 128, *ref) == 1
+    assert L.awq_packed_sizes(256, 500, 128, *ref) == 1     # K not a multiple of g
+    assert L.awq_packed_sizes(256, 512, 128, None, ref[1], ref[2]) == 1
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails before any CUDA call
+
+
+def _lin(L, fn, M=1, N=256, K=512, g=128, ptrs=(FAKE,) * 5, ws=None, ws_bytes=0):
+    x, qw, sc, qz, y = (ctypes.c_void_p(p) for p in ptrs)
+    return getattr(L, fn)(x, qw, sc, qz, y, M, N, K, g, ctypes.c_void_p(ws), ws_bytes, None)
+
+
+@pytest.mark.parametrize("fn", ["w4a16_gemv", "w4a16_gemm", "w4a16_linear"])
+def test_linear_argument_checks(L, fn):
+    assert _lin(L, fn, g=64) == 2
+    assert _lin(L, fn, M=0) == 1
+    assert _lin(L, fn, N=12) == 1          # N % 8 != 0
+    assert _lin(L, fn, K=192) == 1         # K % 128 != 0
+    assert _lin(L, fn, K=0) == 1
+    assert _lin(L, fn, ptrs=(FAKE, 0, FAKE, FAKE, FAKE)) == 1
+    assert _lin(L, fn, ptrs=(FAKE + 4, FAKE, FAKE, FAKE, FAKE)) == 3
+    assert _lin(L, fn, ptrs=(FAKE, FAKE, FAKE, FAKE, FAKE + 2)) == 3
+
+
+def test_pack_and_prep_argument_checks(L):
+    P = ctypes.c_void_p
+    assert L.awq_pack(P(FAKE), None, 256, 512, 64, P(FAKE), P(FAKE), P(FAKE), None) == 2
+    assert L.awq_pack(P(FAKE), None, 256, 500, 128, P(FAKE), P(FAKE), P(FAKE), None) == 1
+    assert L.awq_pack(P(FAKE), None, 0, 512, 128, P(FAKE), P(FAKE), P(FAKE), None) == 1
+    assert L.awq_pack(P(FAKE + 8), None, 256, 512, 128, P(FAKE), P(FAKE), P(FAKE), None) == 3
+    assert L.awq_pack(P(FAKE), P(FAKE + 2), 256, 512, 128, P(FAKE), P(FAKE), P(FAKE), None) == 3
+    assert L.awq_pack(P(FAKE), None, 256, 512, 128, None, P(FAKE), P(FAKE), None) == 1
+    assert L.awq_act_scale(P(FAKE), 0, 512, P(FAKE), None) == 1
+    assert L.awq_act_scale(P(FAKE), 9000, 512, P(FAKE), None) == 1
+    assert L.awq_act_scale(None, 64, 512, P(FAKE), None) == 1
+    assert L.awq_apply_inv_scale(P(FAKE), P(FAKE), 0, 512, P(FAKE), None) == 1
+    assert L.awq_apply_inv_scale(P(FAKE), None, 1, 512, P(FAKE), None) == 1
+
+
+def test_workspace_query_rejects_bad_sizes(L):
+    assert L.w4a16_workspace_bytes(1, 1, 12, 512, 128) == 2**64 - 1
+    assert L.w4a16_workspace_bytes(9, 1, 256, 512, 128) == 2**64 - 1

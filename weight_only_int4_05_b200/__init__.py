@@ -1,0 +1,153 @@
+"""W4A16 group-quantized linear layer (AWQ) for NVIDIA B200 -- Python binding.
+
+Argument marshalling over the C ABI of ``include/awq_w4a16.h`` (``libawq_w4a16.so``): torch supplies
+device memory and the current CUDA stream; every step of the computation runs in the library's CUDA
+kernels.  The functions carry the C entry points' names.
+
+    s  = awq_act_scale(xcal)                    # per-channel AWQ scale, fp16 [K]
+    pw = awq_pack(W, s)                         # packed uint4 weights, fp16 scales, uint4 zeros
+    xp = awq_apply_inv_scale(x, s)              # activations divided by s
+    y  = w4a16_linear(xp, pw)                   # GEMV (decode) or tcgen05 GEMM (prefill) by M
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import NamedTuple, Optional
+
+import torch
+
+from . import _lib
+from ._lib import AwqError, MODE_GEMM, MODE_GEMV, MODE_LINEAR
+
+GROUP = 128
+
+__all__ = [
+    "AwqError", "PackedWeight", "GROUP", "awq_packed_sizes", "awq_act_scale", "awq_apply_inv_scale", "awq_pack",
+    "w4a16_gemv", "w4a16_gemm", "w4a16_linear", "w4a16_gemv_max_m", "w4a16_workspace_bytes",
+    "awq_last_device_status", "reserve_workspace", "lib_path",
+]
+
+
+class PackedWeight(NamedTuple):
+    qweight: torch.Tensor  # int32 [N_pad * K / 8]
+    scales: torch.Tensor   # fp16 [G * N_pad]
+    qzeros: torch.Tensor   # int32 [G * N_pad / 8]
+    N: int
+    K: int
+
+
+def lib_path() -> str:
+    return _lib.lib_path()
+
+
+def _p(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda_fp16(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda or t.dtype != torch.float16 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA float16 tensor")
+
+
+def awq_packed_sizes(N: int, K: int, g: int = GROUP):
+    L = _lib.load()
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _lib.check(L.awq_packed_sizes(N, K, g, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)), "awq_packed_sizes")
+    return a.value, b.value, c.value
+
+
+def awq_act_scale(xcal: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need_cuda_fp16(xcal, "xcal")
+    R, K = xcal.shape
+    s = torch.empty(K, dtype=torch.float16, device=xcal.device) if out is None else out
+    L = _lib.load()
+    _lib.check(L.awq_act_scale(_p(xcal), R, K, _p(s), _stream(xcal.device)), "awq_act_scale")
+    return s
+
+
+def awq_apply_inv_scale(x: torch.Tensor, s: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need_cuda_fp16(x, "x")
+    _need_cuda_fp16(s, "s")
+    M, K = x.shape
+    xp = torch.empty_like(x) if out is None else out
+    L = _lib.load()
+    _lib.check(L.awq_apply_inv_scale(_p(x), _p(s), M, K, _p(xp), _stream(x.device)), "awq_apply_inv_scale")
+    return xp
+
+
+def awq_pack(W: torch.Tensor, s: Optional[torch.Tensor] = None, g: int = GROUP) -> PackedWeight:
+    _need_cuda_fp16(W, "W")
+    if s is not None:
+        _need_cuda_fp16(s, "s")
+    N, K = W.shape
+    qb, sb, zb = awq_packed_sizes(N, K, g)
+    dev = W.device
+    qw = torch.empty(qb // 4, dtype=torch.int32, device=dev)
+    sc = torch.empty(sb // 2, dtype=torch.float16, device=dev)
+    qz = torch.empty(zb // 4, dtype=torch.int32, device=dev)
+    L = _lib.load()
+    _lib.check(L.awq_pack(_p(W), _p(s), N, K, g, _p(qw), _p(sc), _p(qz), _stream(dev)), "awq_pack")
+    return PackedWeight(qw, sc, qz, N, K)
+
+
+# ---- workspace: one zero-initialised buffer per device, grown on demand (the kernels leave it
+# ready for the next call).  Reserve the largest size before capturing CUDA graphs.
+_workspaces: dict = {}
+
+
+def w4a16_workspace_bytes(mode: int, M: int, N: int, K: int, g: int = GROUP) -> int:
+    return int(_lib.load().w4a16_workspace_bytes(mode, M, N, K, g))
+
+
+def reserve_workspace(nbytes: int, device=None) -> torch.Tensor:
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
+        _workspaces[key] = ws
+    return ws
+
+
+def _linear_call(fn_name: str, mode: int, x: torch.Tensor, pw: PackedWeight, out, workspace, g: int):
+    _need_cuda_fp16(x, "x")
+    M, K = x.shape
+    if K != pw.K:
+        raise ValueError(f"x has K={K}, weight has K={pw.K}")
+    N = pw.N
+    y = torch.empty((M, N), dtype=torch.float16, device=x.device) if out is None else out
+    need = w4a16_workspace_bytes(mode, M, N, K, g)
+    if need == 2**64 - 1:
+        raise AwqError(fn_name, 1)
+    ws = workspace if workspace is not None else (reserve_workspace(need, x.device) if need > 0 else None)
+    L = _lib.load()
+    fn = getattr(L, fn_name)
+    st = fn(_p(x), _p(pw.qweight), _p(pw.scales), _p(pw.qzeros), _p(y), M, N, K, g, _p(ws),
+            0 if ws is None else ws.numel() * ws.element_size(), _stream(x.device))
+    _lib.check(st, fn_name)
+    return y
+
+
+def w4a16_gemv(x, pw: PackedWeight, out=None, workspace=None, g: int = GROUP) -> torch.Tensor:
+    return _linear_call("w4a16_gemv", MODE_GEMV, x, pw, out, workspace, g)
+
+
+def w4a16_gemm(x, pw: PackedWeight, out=None, workspace=None, g: int = GROUP) -> torch.Tensor:
+    return _linear_call("w4a16_gemm", MODE_GEMM, x, pw, out, workspace, g)
+
+
+def w4a16_linear(x, pw: PackedWeight, out=None, workspace=None, g: int = GROUP) -> torch.Tensor:
+    return _linear_call("w4a16_linear", MODE_LINEAR, x, pw, out, workspace, g)
+
+
+def w4a16_gemv_max_m(N: int, K: int) -> int:
+    return int(_lib.load().w4a16_gemv_max_m(N, K))
+
+
+def awq_last_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    st = torch.cuda.current_stream() if stream is None else stream
+    return int(_lib.load().awq_last_device_status(ctypes.c_void_p(st.cuda_stream)))

@@ -1,0 +1,176 @@
+// api.cu -- the extern "C" entry points declared in include/awq_w4a16.h.
+//
+// Every entry point validates its arguments on the host and returns a status without launching
+// anything when they are out of range; otherwise it enqueues the kernels on the caller's stream and
+// returns.  No entry point allocates device memory.  The device status word (set by kernels whose
+// bounded waits run out) is a file-scope __device__ variable; its address is looked up once per device.
+#include <stdint.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace awq {
+
+__device__ unsigned g_device_status = 0u;
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = v > 0 ? v : 1;
+  }
+  return cached[dev];
+}
+
+static unsigned* device_status_ptr() {
+  static unsigned* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (cached[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    cached[dev] = static_cast<unsigned*>(p);
+  }
+  return cached[dev];
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxN = 1 << 21;   // packed row blocks index grid.y of the pack kernel
+constexpr int kMaxK = 1 << 20;
+
+static awq_status check_linear(const uint16_t* x, const uint32_t* qw, const uint16_t* sc, const uint32_t* qz,
+                               const uint16_t* y, int M, int N, int K, int g) {
+  if (g != 128) return AWQ_ERR_UNSUPPORTED;
+  if (M < 1 || N < 1 || K < 128 || K % 128 != 0 || N % 8 != 0 || N > kMaxN || K > kMaxK)
+    return AWQ_ERR_INVALID_ARG;
+  if (!x || !qw || !sc || !qz || !y) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(qw) || !aligned16(sc) || !aligned16(qz) || !aligned16(y))
+    return AWQ_ERR_MISALIGNED;
+  return AWQ_OK;
+}
+
+}  // namespace awq
+
+using namespace awq;
+
+extern "C" {
+
+const char* awq_status_string(awq_status st) {
+  switch (st) {
+    case AWQ_OK: return "AWQ_OK";
+    case AWQ_ERR_INVALID_ARG: return "AWQ_ERR_INVALID_ARG";
+    case AWQ_ERR_UNSUPPORTED: return "AWQ_ERR_UNSUPPORTED";
+    case AWQ_ERR_MISALIGNED: return "AWQ_ERR_MISALIGNED";
+    case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA";
+    case AWQ_ERR_DEVICE_TIMEOUT: return "AWQ_ERR_DEVICE_TIMEOUT";
+    case AWQ_ERR_WORKSPACE: return "AWQ_ERR_WORKSPACE";
+  }
+  return "AWQ_ERR_UNKNOWN";
+}
+
+int awq_version(void) { return 100; }
+
+awq_status awq_packed_sizes(int N, int K, int g, size_t* qweight_bytes, size_t* scales_bytes,
+                            size_t* qzeros_bytes) {
+  if (!qweight_bytes || !scales_bytes || !qzeros_bytes) return AWQ_ERR_INVALID_ARG;
+  if (g != 128) return AWQ_ERR_UNSUPPORTED;
+  if (N < 1 || K < 1 || K % g != 0 || N > kMaxN || K > kMaxK) return AWQ_ERR_INVALID_ARG;
+  const size_t Np = (size_t)(N + 31) / 32 * 32;
+  const size_t G = (size_t)K / 128;
+  *qweight_bytes = Np * (size_t)K / 2;
+  *scales_bytes = G * Np * 2;
+  *qzeros_bytes = G * Np / 2;
+  return AWQ_OK;
+}
+
+awq_status awq_act_scale(const uint16_t* d_xcal, int R, int K, uint16_t* d_s, awq_stream_t stream) {
+  if (R < 1 || R > 8192 || K < 1 || K > kMaxK || !d_xcal || !d_s) return AWQ_ERR_INVALID_ARG;
+  return prep_act_scale_launch(d_xcal, R, K, d_s, reinterpret_cast<cudaStream_t>(stream));
+}
+
+awq_status awq_apply_inv_scale(const uint16_t* d_x, const uint16_t* d_s, int M, int K, uint16_t* d_xp,
+                               awq_stream_t stream) {
+  if (M < 1 || K < 1 || K > kMaxK || !d_x || !d_s || !d_xp) return AWQ_ERR_INVALID_ARG;
+  return prep_inv_scale_launch(d_x, d_s, M, K, d_xp, reinterpret_cast<cudaStream_t>(stream));
+}
+
+awq_status awq_pack(const uint16_t* d_W, const uint16_t* d_s, int N, int K, int g, uint32_t* d_qweight,
+                    uint16_t* d_scales, uint32_t* d_qzeros, awq_stream_t stream) {
+  if (g != 128) return AWQ_ERR_UNSUPPORTED;
+  if (N < 1 || K < 1 || K % 128 != 0 || N > kMaxN || K > kMaxK) return AWQ_ERR_INVALID_ARG;
+  if (!d_W || !d_qweight || !d_scales || !d_qzeros) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(d_W) || (d_s && !aligned16(d_s)) || !aligned16(d_qweight) || !aligned16(d_scales) ||
+      !aligned16(d_qzeros))
+    return AWQ_ERR_MISALIGNED;
+  return pack_launch(d_W, d_s, N, K, d_qweight, d_scales, d_qzeros, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t w4a16_workspace_bytes(int mode, int M, int N, int K, int g) {
+  if (g != 128 || M < 1 || N < 1 || K < 128 || K % 128 != 0 || N % 8 != 0 || N > kMaxN || K > kMaxK)
+    return SIZE_MAX;
+  switch (mode) {
+    case AWQ_MODE_GEMV: return gemv_workspace_bytes(M, N, K);
+    case AWQ_MODE_GEMM: return gemm_workspace_bytes(M, N, K);
+    case AWQ_MODE_LINEAR:
+      return M <= w4a16_gemv_max_m(N, K) ? gemv_workspace_bytes(M, N, K) : gemm_workspace_bytes(M, N, K);
+    default: return SIZE_MAX;
+  }
+}
+
+awq_status w4a16_gemv(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                      const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g, void* d_workspace,
+                      size_t workspace_bytes, awq_stream_t stream) {
+  awq_status st = check_linear(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g);
+  if (st != AWQ_OK) return st;
+  if (d_workspace && !aligned16(d_workspace)) return AWQ_ERR_MISALIGNED;
+  return gemv_launch(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, d_workspace, workspace_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+awq_status w4a16_gemm(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                      const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g, void* d_workspace,
+                      size_t workspace_bytes, awq_stream_t stream) {
+  awq_status st = check_linear(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g);
+  if (st != AWQ_OK) return st;
+  if (d_workspace && !aligned16(d_workspace)) return AWQ_ERR_MISALIGNED;
+  if (workspace_bytes < gemm_workspace_bytes(M, N, K)) return AWQ_ERR_WORKSPACE;
+  unsigned* status = device_status_ptr();
+  if (status == nullptr) return AWQ_ERR_CUDA;
+  return gemm_launch(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, d_workspace, workspace_bytes, status,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w4a16_gemv_max_m(int N, int K) {
+  (void)N;
+  (void)K;
+  return 8;
+}
+
+awq_status w4a16_linear(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                        const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g, void* d_workspace,
+                        size_t workspace_bytes, awq_stream_t stream) {
+  if (M >= 1 && M <= w4a16_gemv_max_m(N, K))
+    return w4a16_gemv(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g, d_workspace, workspace_bytes, stream);
+  return w4a16_gemm(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g, d_workspace, workspace_bytes, stream);
+}
+
+awq_status awq_last_device_status(awq_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return AWQ_ERR_CUDA;
+  unsigned* p = device_status_ptr();
+  if (p == nullptr) return AWQ_ERR_CUDA;
+  unsigned v = 0u;
+  if (cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (v != 0u) {
+    const unsigned zero = 0u;
+    if (cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return AWQ_ERR_CUDA;
+    return AWQ_ERR_DEVICE_TIMEOUT;
+  }
+  return AWQ_OK;
+}
+
+}  // extern "C"
