@@ -1,0 +1,540 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A16 AWQ linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Metric: W4A16 GEMV HBM GB/s (% of peak) at M=1; GEMM TFLOP/s at M=2048.
+  * value (first head): one step = one synthetic 8B-class decode token through the full stack of
+    32 layers x 7 W4A16 linears (q, k, v, o, gate, up, down with Llama-3-8B shapes) at M=1, run back to
+    back on one stream through w4a16_linear (GEMV mode), captured as one CUDA graph with programmatic
+    dependent launch.  GB/s = algorithmic bytes per step (packed weights + scales + zeros + x' + y) over
+    the device time of the step.  3.63 GB per step, far larger than the 126 MB L2, so every step streams
+    from HBM.
+  * gemm (second head): the three prefill shapes at M=2048 tokens through w4a16_gemm, TFLOP/s =
+    2 M N K / device time (one step = the three shapes back to back, ~250 MB of operands > L2).
+Inputs are synthetic (seeded torch CUDA generator; W ~ N(0, 0.02^2), activations N(0,1) with 1% of the
+channels x20), quantized on the device with awq_act_scale / awq_pack / awq_apply_inv_scale.
+With N > 1 GPUs every rank runs an independent replica (the layer needs no exchange); value is the
+bytes of all ranks over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "W4A16 GEMV HBM GB/s (% of peak) at M=1; GEMM TFLOP/s at M=2048"
+DECODE_SHAPES = [("q", 4096, 4096), ("k", 4096, 1024), ("v", 4096, 1024), ("o", 4096, 4096),
+                 ("gate", 4096, 14336), ("up", 4096, 14336), ("down", 14336, 4096)]  # (name, K, N)
+LAYERS = 32
+PREFILL_SHAPES = [(4096, 14336), (14336, 4096), (4096, 4096)]  # (K, N)
+PREFILL_M = 2048
+BYTES_PER_WEIGHT = 0.5 + 2.0 / 128 + 0.5 / 128
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_GEMV = os.path.join(ROOT, "profiles", "gemv_kernel_decode_stack.md")
+PROFILE_GEMM = os.path.join(ROOT, "profiles", "gemm_kernel_prefill_m2048.md")
+
+
+def gemv_bytes(M, N, K):
+    """Algorithmic bytes of one W4A16 linear: packed weight + scales + zeros, x' and y."""
+    return N * K * BYTES_PER_WEIGHT + 2 * M * K + 2 * M * N
+
+
+def decode_step_bytes(M=1):
+    return LAYERS * sum(gemv_bytes(M, N, K) for _, K, N in DECODE_SHAPES)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+GEMV_SOURCES = ["weight_only_int4_05_b200/csrc/gemv.cu", "weight_only_int4_05_b200/csrc/common.cuh"]
+GEMM_SOURCES = ["weight_only_int4_05_b200/csrc/gemm.cu", "weight_only_int4_05_b200/csrc/common.cuh"]
+
+
+def profiled_traffic(profile_path, sources):
+    """DRAM bytes per launch recorded by an ncu capture, or None when the kernel changed since."""
+    try:
+        text = open(profile_path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    m_val = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_val or m_hash.group(1) != source_hash(sources):
+        return None
+    return float(m_val.group(1))
+
+
+# ------------------------------------------------------------------------------- distributed plumbing
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_max(value: float, group_backend_device=None) -> float:
+    """Maximum of `value` over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=group_backend_device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate_value(bytes_per_rank_step: float, steps: int, world: int, max_seconds: float) -> float:
+    """Whole-job GB/s: the bytes every rank processed over the slowest rank's time."""
+    return bytes_per_rank_step * steps * world / max_seconds / 1e9
+
+
+# ------------------------------------------------------------------------------- clocks sampling
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t is not None:
+            self._t.join(timeout=2)
+        return summarize_clock_lines(self.lines)
+
+
+def summarize_clock_lines(lines):
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    sm, smax, reasons, power = [], [], set(), []
+    for ln in lines:
+        parts = [p.strip() for p in ln.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            smax.append(float(parts[2]))
+            power.append(float(parts[3]))
+        except ValueError:
+            continue
+        for name, val in zip(names, parts[5:9]):
+            if val.lower().startswith("active"):
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+            "reasons": sorted(reasons), "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------------------- GPU workloads
+class DecodeStack:
+    """32 layers x 7 packed linears, inputs x' and outputs y resident in HBM, one CUDA graph per step."""
+
+    def __init__(self, device, seed=0, M=1, layers=LAYERS):
+        import torch
+        import synth
+        import weight_only_int4_05_b200 as W4
+
+        self.W4, self.torch, self.device, self.M = W4, torch, device, M
+        self.entries = []  # (packed weight, x' view, y view)
+        shapes = [(li, name, K, N) for li in range(layers) for (name, K, N) in DECODE_SHAPES]
+        self.h2d_elems = sum(M * K for _, _, K, _ in shapes)
+        self.d2h_elems = sum(M * N for _, _, _, N in shapes)
+        self.x_all = torch.empty(self.h2d_elems, dtype=torch.float16, device=device)
+        self.y_all = torch.empty(self.d2h_elems, dtype=torch.float16, device=device)
+        xo = yo = 0
+        for idx, (li, name, K, N) in enumerate(shapes):
+            tid = synth.tensor_id(2, li, DECODE_SHAPES.index((name, K, N)), 0)
+            Wt, xcal, x = synth.device_linear_inputs(seed, tid, M, N, K, device)
+            s = W4.awq_act_scale(xcal)
+            pw = W4.awq_pack(Wt, s)
+            xv = self.x_all[xo:xo + M * K].view(M, K)
+            W4.awq_apply_inv_scale(x, s, out=xv)
+            yv = self.y_all[yo:yo + M * N].view(M, N)
+            self.entries.append((pw, xv, yv, K, N))
+            xo += M * K
+            yo += M * N
+            del Wt, xcal, x
+        self.launches_per_step = sum(self._launches(K, N) for _, _, _, K, N in self.entries)
+        need = max(W4.w4a16_workspace_bytes(W4.MODE_LINEAR, M, N, K) for _, _, _, K, N in self.entries)
+        W4.reserve_workspace(need, device)
+        torch.cuda.synchronize(device)
+        self.graph = None
+
+    def _launches(self, K, N):
+        W4 = self.W4
+        if self.M <= W4.w4a16_gemv_max_m(N, K):
+            return (self.M + 7) // 8 if self.M > 4 else 1
+        return 1
+
+    def eager_step(self):
+        for pw, xv, yv, _, _ in self.entries:
+            self.W4.w4a16_linear(xv, pw, out=yv)
+
+    def capture(self):
+        torch = self.torch
+        s = torch.cuda.Stream(self.device)
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(s):
+            self.eager_step()  # warm caches (occupancy queries, workspace) outside the capture
+        torch.cuda.current_stream(self.device).wait_stream(s)
+        torch.cuda.synchronize(self.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.eager_step()
+        torch.cuda.synchronize(self.device)
+
+    def step(self):
+        self.graph.replay()
+
+    def bytes_per_step(self):
+        return sum(gemv_bytes(self.M, N, K) for _, _, _, K, N in self.entries)
+
+
+class PrefillGemm:
+    """The three M=2048 prefill shapes, one CUDA graph per step (all three back to back)."""
+
+    def __init__(self, device, seed=0, M=PREFILL_M):
+        import torch
+        import synth
+        import weight_only_int4_05_b200 as W4
+
+        self.W4, self.torch, self.device, self.M = W4, torch, device, M
+        self.entries = []
+        for i, (K, N) in enumerate(PREFILL_SHAPES):
+            Wt, xcal, x = synth.device_linear_inputs(seed, synth.tensor_id(3, 0, i, 0), M, N, K, device)
+            s = W4.awq_act_scale(xcal)
+            pw = W4.awq_pack(Wt, s)
+            xp = W4.awq_apply_inv_scale(x, s)
+            y = torch.empty((M, N), dtype=torch.float16, device=device)
+            self.entries.append((pw, xp, y, K, N))
+            del Wt, xcal, x
+        need = max(W4.w4a16_workspace_bytes(W4.MODE_GEMM, M, N, K) for _, _, _, K, N in self.entries)
+        W4.reserve_workspace(need, device)
+        torch.cuda.synchronize(device)
+
+    def eager_step(self):
+        for pw, xp, y, _, _ in self.entries:
+            self.W4.w4a16_gemm(xp, pw, out=y)
+
+    def capture(self):
+        torch = self.torch
+        self.eager_step()
+        torch.cuda.synchronize(self.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.eager_step()
+        torch.cuda.synchronize(self.device)
+
+    def step(self):
+        self.graph.replay()
+
+    def flops_per_step(self):
+        return sum(2.0 * self.M * N * K for _, _, _, K, N in self.entries)
+
+
+def time_steps(step_fn, steps, warmup, device, sampler=None):
+    """Device time of `steps` calls of step_fn (CUDA events on the current stream), max over ranks."""
+    import torch
+
+    for _ in range(warmup):
+        step_fn()
+    barrier(device)
+    torch.cuda.synchronize(device)
+    if sampler is not None:
+        sampler.start()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(steps):
+        step_fn()
+    ev1.record()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop() if sampler is not None else None
+    seconds = ev0.elapsed_time(ev1) / 1e3
+    return reduce_max(seconds, device), clocks
+
+
+def e2e_decode(stack, steps, warmup, device):
+    """Same metric through the public API with host buffers: every step copies all 224 x' from pinned
+    host memory, runs the graph, and reads all y back to pinned host memory."""
+    import torch
+
+    x_host = stack.x_all.cpu().pin_memory()
+    y_host = torch.empty(stack.y_all.shape, dtype=torch.float16).pin_memory()
+
+    def step():
+        stack.x_all.copy_(x_host, non_blocking=True)
+        stack.step()
+        y_host.copy_(stack.y_all, non_blocking=True)
+
+    seconds, _ = time_steps(step, steps, warmup, device)
+    return seconds, x_host.numel() * 2, y_host.numel() * 2
+
+
+# ------------------------------------------------------------------------------- CPU oracle legs
+def oracle_sample_linears(seed=0):
+    """Host inputs for the CPU legs: linears of the decode stack in layer order (host generator)."""
+    import synth
+
+    for li in range(LAYERS):
+        for j, (name, K, N) in enumerate(DECODE_SHAPES):
+            yield li, name, K, N, synth.linear_inputs(seed, 2, li, j, 1, N, K)
+
+
+def oracle_time_linear(d, K, N):
+    """Oracle time (s) of one M=1 linear: every output y[0][n] in fp64 from the quantized weight."""
+    import numpy as np
+    from oracle import oracle as O
+
+    s = O.act_scale(d["xcal"].view(np.uint16))
+    xp = O.inv_scale(d["x"].view(np.uint16), s)
+    q, sc, z = O.quantize(d["W"].view(np.uint16), s)
+    ms = np.zeros(N, np.int32)
+    ns = np.arange(N, dtype=np.int32)
+    t0 = time.perf_counter()
+    O.linear_pairs_f64(xp, q, sc, z, ms, ns)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(budget_s=12.0):
+    """The oracle as it stands, single-threaded on this host, on the first linears of the decode stack
+    until about `budget_s` seconds of oracle time; GB/s of the same algorithmic bytes."""
+    total_t = total_b = 0.0
+    names = []
+    for li, name, K, N, d in oracle_sample_linears():
+        total_t += oracle_time_linear(d, K, N)
+        total_b += gemv_bytes(1, N, K)
+        names.append(f"L{li}.{name}")
+        if total_t >= budget_s:
+            break
+    return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(names)} linears of the M=1 decode stack ({names[0]}..{names[-1]}), "
+                      f"{total_b / 1e6:.1f} MB of packed weight, {total_t:.1f} s of single-thread oracle time"}
+
+
+REF_ROWS_PER_STEP = 256
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle on this host's cores.  One step = 256 outputs of the next M=1 linear
+    of the decode stack (layer 0's q, k, v, o, gate, up, down, cycling) -- a bounded sample of the decode
+    workload; GB/s counts the algorithmic bytes of exactly those outputs."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import numpy as np
+    from oracle import oracle as O
+
+    prepared = []
+    for li, name, K, N, d in oracle_sample_linears():
+        s = O.act_scale(d["xcal"].view(np.uint16))
+        xp = O.inv_scale(d["x"].view(np.uint16), s)
+        q, sc, z = O.quantize(d["W"].view(np.uint16), s)
+        prepared.append((K, N, xp, q, sc, z))
+        if len(prepared) >= len(DECODE_SHAPES):
+            break
+    rows = REF_ROWS_PER_STEP
+
+    def step(i):
+        K, N, xp, q, sc, z = prepared[i % len(prepared)]
+        ns = (np.arange(rows, dtype=np.int32) + (i * rows)) % N
+        ms = np.zeros(rows, np.int32)
+        t0 = time.perf_counter()
+        O.linear_pairs_f64(xp, q, sc, z, ms, ns)
+        return time.perf_counter() - t0, rows * K * BYTES_PER_WEIGHT + 2 * K + 2 * rows
+
+    for i in range(args.warmup):
+        step(i)
+    tt = bb = 0.0
+    for i in range(args.steps):
+        t, b = step(i)
+        tt += t
+        bb += b
+    value = bb / tt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "decode stack (32 layers x 7 Llama-3-8B-shaped W4A16 linears, M=1); each step "
+                                   "a bounded sample: 256 outputs of the next linear of layer 0",
+                       "M": 1, "rows_per_step": rows},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{args.steps} steps x {rows} outputs, {bb / 1e6:.1f} MB of packed weight"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------------------- our arm
+def gpu_uuid_id(device):
+    import torch
+
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        return str(device.index)
+
+
+def run_gpu(args):
+    import datetime
+
+    import torch
+
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    import weight_only_int4_05_b200 as W4
+
+    W4._lib.load()  # fails loudly if the CUDA library is missing
+    peaks, peak_src = load_peaks()
+
+    # ---- head 1: decode stack, GEMV mode
+    stack = DecodeStack(device)
+    stack.capture()
+    sampler = ClockSampler(gpu_uuid_id(device))
+    seconds, clocks = time_steps(stack.step, args.steps, args.warmup, device, sampler)
+    bytes_step = stack.bytes_per_step()
+    value = aggregate_value(bytes_step, args.steps, world, seconds)
+    per_gpu = value / world
+    launches = stack.launches_per_step
+    gemv_traffic = profiled_traffic(PROFILE_GEMV, GEMV_SOURCES)
+    roofline = {"bound": "hbm", "achieved": per_gpu, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": per_gpu / peaks["hbm_gbs"], "traffic": gemv_traffic,
+                "kernel": "gemv_kernel<1>", "peak_source": peak_src,
+                "bytes_per_launch": bytes_step / launches, "launch_us": seconds / args.steps / launches * 1e6}
+
+    # ---- e2e through the public API with host buffers
+    e2e_steps = max(3, args.steps // 4)
+    e2e_s, h2d, d2h = e2e_decode(stack, e2e_steps, max(3, args.warmup // 4), device)
+    e2e_value = aggregate_value(bytes_step, e2e_steps, world, e2e_s)
+
+    # ---- head 2: prefill GEMM at M=2048
+    del stack
+    torch.cuda.empty_cache()
+    pre = PrefillGemm(device)
+    pre.capture()
+    g_steps = max(5, min(100, args.steps // 20))
+    g_sampler = ClockSampler(gpu_uuid_id(device))
+    g_seconds, g_clocks = time_steps(pre.step, g_steps, max(3, args.warmup // 4), device, g_sampler)
+    tflops = pre.flops_per_step() * g_steps * world / g_seconds / 1e12
+    g_per_gpu = tflops / world
+    gemm = {"value": tflops, "unit": "TFLOP/s", "ms_per_step": g_seconds / g_steps * 1e3, "steps": g_steps,
+            "workload": "prefill GEMM M=2048: (K,N) = (4096,14336), (14336,4096), (4096,4096), one step = all three",
+            "gpu_launches": 3 * g_steps, "clocks": g_clocks,
+            "roofline": {"bound": "tensor", "achieved": g_per_gpu, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": g_per_gpu / peaks["bf16_tflops"],
+                         "frac_of_sustained": g_per_gpu / peaks["bf16_tflops_sustained"],
+                         "traffic": profiled_traffic(PROFILE_GEMM, GEMM_SOURCES), "kernel": "gemm_kernel",
+                         "peak_source": peak_src + " (dense bf16 burst; fp16 runs at the bf16 tensor rate)"}}
+
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": seconds / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "pct_of_peak": 100.0 * per_gpu / peaks["hbm_gbs"],
+            "config": {"workload": "decode stack: 32 layers x 7 W4A16 linears (Llama-3-8B shapes: q/o 4096->4096, "
+                                   "k/v 4096->1024, gate/up 4096->14336, down 14336->4096), M=1, one token per step",
+                       "M": 1, "layers": LAYERS, "group_size": 128, "bytes_per_step": bytes_step,
+                       "l2": "inputs larger than L2 (3.63 GB of packed weights per step)",
+                       "accumulate": "f32", "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "roofline": roofline, "gpu_launches": launches * args.steps, "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "gemm": gemm}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    status = W4.awq_last_device_status()
+    if status != 0:
+        line["device_status"] = status
+    if world > 1:
+        import torch.distributed as dist
+
+        barrier(device)
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

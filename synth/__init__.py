@@ -53,17 +53,78 @@ def stream_u64(key: np.uint64, start: int, count: int) -> np.ndarray:
         return _splitmix64(idx + key)
 
 
-def standard_normal(key: np.uint64, count: int, chunk: int = 1 << 22) -> np.ndarray:
+class _NormalStream:
+    """Standard normals of one stream, produced chunk by chunk in reused buffers (large fresh
+    allocations are what makes naive numpy generation slow)."""
+
+    def __init__(self, key: np.uint64, chunk: int = 1 << 20):
+        self.key = key
+        self.chunk = chunk
+        self.ctr = np.empty(2 * chunk, np.uint64)
+        self.tmp = np.empty(2 * chunk, np.uint64)
+        self.u1 = np.empty(chunk, np.float64)
+        self.u2 = np.empty(chunk, np.float64)
+        self.base = np.arange(2 * chunk, dtype=np.uint64)
+
+    def block(self, start: int, c: int) -> np.ndarray:
+        """Normals for elements start .. start+c-1 (c <= chunk), as a view of an internal buffer."""
+        ctr, tmp = self.ctr[:2 * c], self.tmp[:2 * c]
+        with np.errstate(over="ignore"):
+            np.add(self.base[:2 * c], self.key + np.uint64(2 * start), out=ctr)
+            np.add(ctr, _GAMMA, out=ctr)                       # splitmix64, in place
+            np.right_shift(ctr, np.uint64(30), out=tmp)
+            np.bitwise_xor(ctr, tmp, out=ctr)
+            np.multiply(ctr, _C1, out=ctr)
+            np.right_shift(ctr, np.uint64(27), out=tmp)
+            np.bitwise_xor(ctr, tmp, out=ctr)
+            np.multiply(ctr, _C2, out=ctr)
+            np.right_shift(ctr, np.uint64(31), out=tmp)
+            np.bitwise_xor(ctr, tmp, out=ctr)
+        u1, u2 = self.u1[:c], self.u2[:c]
+        np.right_shift(ctr[0::2], np.uint64(11), out=tmp[:c])
+        np.add(tmp[:c], np.uint64(1), out=tmp[:c])
+        np.multiply(tmp[:c], 2.0 ** -53, out=u1)              # (0, 1]
+        np.right_shift(ctr[1::2], np.uint64(11), out=tmp[:c])
+        np.multiply(tmp[:c], 2.0 ** -53, out=u2)              # [0, 1)
+        np.log(u1, out=u1)
+        np.multiply(u1, -2.0, out=u1)
+        np.sqrt(u1, out=u1)
+        np.multiply(u2, 2.0 * np.pi, out=u2)
+        np.cos(u2, out=u2)
+        np.multiply(u1, u2, out=u1)
+        return u1
+
+
+def standard_normal(key: np.uint64, count: int, chunk: int = 1 << 20) -> np.ndarray:
     """count standard normals (fp64) from stream `key`; element i uses stream values 2i and 2i+1."""
     out = np.empty(count, np.float64)
+    ns = _NormalStream(key, chunk)
     for s in range(0, count, chunk):
         c = min(chunk, count - s)
-        u = stream_u64(key, 2 * s, 2 * c)
-        a, b = u[0::2], u[1::2]
-        u1 = ((a >> np.uint64(11)).astype(np.float64) + 1.0) * (2.0 ** -53)
-        u2 = (b >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
-        out[s:s + c] = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+        out[s:s + c] = ns.block(s, c)
     return out
+
+
+def _fp16_normals(key: np.uint64, rows: int, cols: int, row_gain=None, sigma: float = 1.0,
+                  chunk: int = 1 << 20) -> np.ndarray:
+    """fp16 [rows][cols] = fp16(sigma * z * gain[col]) with z the stream's normals in row-major order."""
+    out = np.empty(rows * cols, np.float16)
+    ns = _NormalStream(key, chunk)
+    total = rows * cols
+    gain = None
+    if row_gain is not None:
+        reps = (chunk + cols - 1) // cols + 1
+        gain = np.tile(row_gain.astype(np.float64) * sigma, reps)
+    for s in range(0, total, chunk):
+        c = min(chunk, total - s)
+        z = ns.block(s, c)
+        if gain is not None:
+            off = s % cols
+            np.multiply(z, gain[off:off + c], out=z)
+        elif sigma != 1.0:
+            np.multiply(z, sigma, out=z)
+        out[s:s + c] = z
+    return out.reshape(rows, cols)
 
 
 def tensor_id(config: int, layer: int, linear: int, kind: int) -> int:
@@ -84,17 +145,16 @@ def outlier_channels(seed: int, K: int, tid: int) -> np.ndarray:
 
 
 def weights(seed: int, tid: int, N: int, K: int) -> np.ndarray:
-    """fp16 W [N][K] ~ N(0, 0.02^2)."""
-    z = standard_normal(stream_key(seed, tid), N * K)
-    return (W_SIGMA * z).astype(np.float16).reshape(N, K)
+    """fp16 W [N][K] = fp16(0.02 z)."""
+    return _fp16_normals(stream_key(seed, tid), N, K, sigma=W_SIGMA)
 
 
 def activations(seed: int, tid: int, rows: int, K: int, outliers: np.ndarray) -> np.ndarray:
-    """fp16 [rows][K] ~ N(0, 1) with the outlier channels scaled by 20 before rounding."""
-    z = standard_normal(stream_key(seed, tid), rows * K).reshape(rows, K)
+    """fp16 [rows][K] = fp16(z), and fp16(20 z) in the outlier channels."""
+    gain = np.ones(K, np.float64)
     if len(outliers):
-        z[:, outliers] *= OUTLIER_GAIN
-    return z.astype(np.float16)
+        gain[outliers] = OUTLIER_GAIN
+    return _fp16_normals(stream_key(seed, tid), rows, K, row_gain=gain)
 
 
 def linear_inputs(seed: int, config: int, layer: int, linear: int, M: int, N: int, K: int) -> dict:
