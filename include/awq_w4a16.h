@@ -165,6 +165,18 @@ awq_status w4a16_gemm(const uint16_t* d_x, const uint32_t* d_qweight, const uint
                       const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
                       void* d_workspace, size_t workspace_bytes, awq_stream_t stream);
 
+/* w4a16_gemv_noalloc -- the same computation as w4a16_gemv for callers that cannot allocate device
+ * memory (e.g. a plug-in whose host framework owns every allocation, or a serving loop whose memory
+ * budget is fixed at start-up).  The pages have no counterpart: this is a deployment convenience.
+ * The split-K scratch is a library-owned static device array of 8 MiB per device (held by every GPU
+ * that loads the library until exit); sizes whose scratch would exceed it return AWQ_ERR_WORKSPACE.
+ * Nothing is allocated: the call clears the array's counters with cudaMemsetAsync and launches the
+ * GEMV.  The first call on a device looks up the array's address (cudaGetSymbolAddress); make it
+ * before any stream capture.  All calls share the array: calls that overlap on the GPU race. */
+awq_status w4a16_gemv_noalloc(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                              const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
+                              awq_stream_t stream);
+
 /* w4a16_linear -- picks GEMV when M <= w4a16_gemv_max_m(N, K), GEMM otherwise, and calls it. */
 awq_status w4a16_linear(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
                         const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,

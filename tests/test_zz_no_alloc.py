@@ -1,0 +1,58 @@
+"""w4a16_gemv_noalloc, the GEMV entry point for callers that cannot allocate device memory (its
+split-K scratch is a static device array owned by the library).  Called through the C ABI and checked
+against w4a16_gemv with the layer tolerance of the other tests, on two calls in a row (the second
+call finds the first call's leftovers in the shared array).  Runs alone or after the other tests."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from weight_only_int4_05_b200 import _lib, build as libbuild
+import weight_only_int4_05_b200 as W4
+from helpers import assert_within_tolerance
+
+pytestmark = pytest.mark.gpu
+
+
+def _packed(N, K, seed):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    Wt = (torch.randn((N, K), generator=g, device="cuda") * 0.02).half()
+    s = (torch.rand((K,), generator=g, device="cuda") + 0.5).half()
+    x = torch.randn((8, K), generator=g, device="cuda").half()
+    return W4.awq_pack(Wt, s), x
+
+
+def _call_noalloc(L, x, pw, y):
+    M, K = x.shape
+    P = ctypes.c_void_p
+    stream = P(torch.cuda.current_stream().cuda_stream)
+    return L.w4a16_gemv_noalloc(P(x.data_ptr()), P(pw.qweight.data_ptr()), P(pw.scales.data_ptr()),
+                                P(pw.qzeros.data_ptr()), P(y.data_ptr()), M, pw.N, K, 128, stream)
+
+
+def test_noalloc_matches_gemv_on_two_calls_in_a_row():
+    libbuild.build()
+    L = _lib.load()
+    torch.cuda.set_device(0)
+    cases = [(_packed(14336, 4096, 1), 1), (_packed(264, 1152, 2), 5)]  # split-K, then a ragged shape
+    for (pw, x_all), M in cases:
+        x = x_all[:M].contiguous()
+        y = torch.empty((M, pw.N), dtype=torch.float16, device="cuda")
+        assert _call_noalloc(L, x, pw, y) == 0
+        y_ref = W4.w4a16_gemv(x, pw)
+        torch.cuda.synchronize()
+        assert_within_tolerance(y.float().cpu().numpy(), y_ref.float().cpu().numpy().astype(np.float64),
+                                f"noalloc N={pw.N}")
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    libbuild.build()
+    L = _lib.load()
+    N, K, M = 131072, 1024, 8
+    need = L.w4a16_workspace_bytes(1, M, N, K, 128)
+    assert need > (8 << 20)
+    FAKE = ctypes.c_void_p(0x10000)
+    st = L.w4a16_gemv_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, M, N, K, 128, None)
+    assert st == 6  # AWQ_ERR_WORKSPACE, nothing launched

@@ -24,7 +24,7 @@ GROUP = 128
 __all__ = [
     "AwqError", "PackedWeight", "GROUP", "awq_packed_sizes", "awq_act_scale", "awq_apply_inv_scale", "awq_pack",
     "w4a16_gemv", "w4a16_gemm", "w4a16_linear", "w4a16_gemv_max_m", "w4a16_workspace_bytes",
-    "awq_last_device_status", "reserve_workspace", "lib_path",
+    "awq_last_device_status", "reserve_workspace", "lib_path", "w4a16_gemv_noalloc",
 ]
 
 
@@ -142,6 +142,21 @@ def w4a16_gemm(x, pw: PackedWeight, out=None, workspace=None, g: int = GROUP) ->
 
 def w4a16_linear(x, pw: PackedWeight, out=None, workspace=None, g: int = GROUP) -> torch.Tensor:
     return _linear_call("w4a16_linear", MODE_LINEAR, x, pw, out, workspace, g)
+
+
+def w4a16_gemv_noalloc(x, pw: PackedWeight, out=None, g: int = GROUP) -> torch.Tensor:
+    """GEMV whose scratch is the library's static device array (no allocation by the library; for
+    callers that cannot allocate device memory).  Overlapping calls on one device race."""
+    _need_cuda_fp16(x, "x")
+    M, K = x.shape
+    if K != pw.K:
+        raise ValueError(f"x has K={K}, weight has K={pw.K}")
+    y = torch.empty((M, pw.N), dtype=torch.float16, device=x.device) if out is None else out
+    L = _lib.load()
+    st = L.w4a16_gemv_noalloc(_p(x), _p(pw.qweight), _p(pw.scales), _p(pw.qzeros), _p(y), M, pw.N, K, g,
+                              _stream(x.device))
+    _lib.check(st, "w4a16_gemv_noalloc")
+    return y
 
 
 def w4a16_gemv_max_m(N: int, K: int) -> int:

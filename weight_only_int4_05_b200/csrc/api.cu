@@ -42,7 +42,7 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 constexpr int kMaxN = 1 << 21;   // packed row blocks index grid.y of the pack kernel
 constexpr int kMaxK = 1 << 20;
 
-static awq_status check_linear(const uint16_t* x, const uint32_t* qw, const uint16_t* sc, const uint32_t* qz,
+awq_status check_linear(const uint16_t* x, const uint32_t* qw, const uint16_t* sc, const uint32_t* qz,
                                const uint16_t* y, int M, int N, int K, int g) {
   if (g != 128) return AWQ_ERR_UNSUPPORTED;
   if (M < 1 || N < 1 || K < 128 || K % 128 != 0 || N % 8 != 0 || N > kMaxN || K > kMaxK)

@@ -16,6 +16,10 @@ constexpr size_t kWorkspaceCounterBytes = 64 * 1024;
 
 int num_sms();  // SM count of the current device (cached per device)
 
+// Host-side argument checks shared by the linear-layer entry points (AWQ_OK when valid).
+awq_status check_linear(const uint16_t* x, const uint32_t* qw, const uint16_t* sc, const uint32_t* qz,
+                        const uint16_t* y, int M, int N, int K, int g);
+
 // Launch with programmatic stream serialization, so the kernel may start while the previous kernel
 // on the stream drains; the kernels order their dependent accesses with griddepcontrol.wait.
 template <typename... KArgs, typename... Args>

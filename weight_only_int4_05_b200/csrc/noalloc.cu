@@ -1,0 +1,51 @@
+// noalloc.cu -- w4a16_gemv_noalloc: the decode GEMV for callers that cannot allocate device memory.
+//
+// Some callers have no way to hand this library a workspace: a plug-in whose host framework owns every
+// device allocation and exposes no allocator to it, or a serving loop with a device-memory budget
+// fixed at start-up that must not allocate per request.  For them the GEMV's split-K scratch lives in
+// a file-scope __device__ array of kNoAllocScratchBytes, which every GPU that loads this library holds
+// until the process exits.
+//
+// The host code below never passes the array's name to a kernel (in host code it is only a stand-in);
+// it looks up the array's device address once per device with cudaGetSymbolAddress and passes that.
+// The first call on each device performs this lookup, so make that first call before any stream
+// capture.  Every call shares the one array and keeps the last call's contents, so each call clears
+// the counters that must start at zero (cudaMemsetAsync, no allocation).  Calls on one device that
+// overlap on the GPU (for example, issued on two streams) race on the array; the caller must order
+// them.  Each device has its own copy of the array.
+#include "common.cuh"
+#include "internal.h"
+
+namespace awq {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+static void* noalloc_scratch_address() {
+  static void* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (cached[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    cached[dev] = p;
+  }
+  return cached[dev];
+}
+
+}  // namespace awq
+
+extern "C" awq_status w4a16_gemv_noalloc(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                                         const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
+                                         awq_stream_t stream) {
+  using namespace awq;
+  awq_status st = check_linear(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g);
+  if (st != AWQ_OK) return st;
+  if (gemv_workspace_bytes(M, N, K) > kNoAllocScratchBytes) return AWQ_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch_address();
+  if (scratch == nullptr) return AWQ_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, kWorkspaceCounterBytes, s) != cudaSuccess) return AWQ_ERR_CUDA;
+  return gemv_launch(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, scratch, kNoAllocScratchBytes, s);
+}
