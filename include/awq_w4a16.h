@@ -45,11 +45,14 @@
  *            i.e. nibble order e = [0, 2, 4, 6, 1, 3, 5, 7].  (Masking the word with 0x000F000F puts
  *            channels e=0,1 in the two 16-bit halves; 0x00F000F0 gives e=2,3; the word shifted right by
  *            8 gives e=4,5 and e=6,7 the same way.)
- *            Consequence: the 32 rows x 128 channels of one (row block, group) are 2048 contiguous
- *            bytes starting at byte (rb * G + g) * 2048.
- *   scales   uint16_t (fp16)[G * N_pad], group major: the scale of row n, group g is scales[g*N_pad + n].
- *   qzeros   uint32_t[G * N_pad / 8], group major: the zero of row n, group g is nibble (n % 8)
- *            (bits 4*(n%8) .. +3) of word qzeros[g*(N_pad/8) + n/8].
+ *            Consequence: the 32 rows x 128 channels of one (row block, group) -- a "unit",
+ *            u = rb * G + g -- are 2048 contiguous bytes starting at byte u * 2048.
+ *   scales   uint16_t (fp16)[G * N_pad], unit major: the scale of row n, group g is
+ *            scales[(rb * G + g) * 32 + r]  (rb = n / 32, r = n % 32): 64 contiguous bytes per unit.
+ *   qzeros   uint32_t[G * N_pad / 8], unit major: the zero of row n, group g is nibble (r % 8)
+ *            (bits 4*(r%8) .. +3) of word qzeros[(rb * G + g) * 4 + r / 8]: 16 bytes per unit.
+ *   So consecutive units are consecutive in all three arrays, and a range of units is one contiguous
+ *   stretch of each array.
  *   Padding rows n = N .. N_pad-1 hold code 0, scale 0 and zero 0 in every array.
  *   Bytes per weight (N a multiple of 32): 0.5 + 2/128 + 0.5/128 = 0.51953.
  *

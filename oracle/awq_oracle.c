@@ -178,8 +178,9 @@ void oracle_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int N, 
       qweight[word] |= (uint32_t)(q[(size_t)n * K + k] & 0xF) << (4 * p);
     }
     for (int gi = 0; gi < G; ++gi) {
-      scales[(size_t)gi * Np + n] = sc[(size_t)n * G + gi];
-      qzeros[(size_t)gi * (Np / 8) + n / 8] |= (uint32_t)(z[(size_t)n * G + gi] & 0xF) << (4 * (n % 8));
+      size_t unit = (size_t)rb * G + gi; /* unit-major scales and zeros */
+      scales[unit * 32 + r] = sc[(size_t)n * G + gi];
+      qzeros[unit * 4 + r / 8] |= (uint32_t)(z[(size_t)n * G + gi] & 0xF) << (4 * (r % 8));
     }
   }
 }
@@ -204,11 +205,16 @@ void oracle_unpack(const uint32_t* qweight, const uint16_t* scales, const uint32
       if (n < N) q[(size_t)n * K + k] = code;
     }
   }
-  for (int gi = 0; gi < G; ++gi)
-    for (int n = 0; n < N; ++n) {
-      sc[(size_t)n * G + gi] = scales[(size_t)gi * Np + n];
-      z[(size_t)n * G + gi] = (uint8_t)((qzeros[(size_t)gi * (Np / 8) + n / 8] >> (4 * (n % 8))) & 0xF);
+  /* scales and zeros: walk the units in storage order */
+  for (size_t unit = 0; unit < (size_t)(Np / 32) * G; ++unit) {
+    int rb = (int)(unit / (size_t)G), gi = (int)(unit % (size_t)G);
+    for (int r = 0; r < 32; ++r) {
+      int n = rb * 32 + r;
+      if (n >= N) continue;
+      sc[(size_t)n * G + gi] = scales[unit * 32 + r];
+      z[(size_t)n * G + gi] = (uint8_t)((qzeros[unit * 4 + r / 8] >> (4 * (r % 8))) & 0xF);
     }
+  }
 }
 
 /* ------------------------------------------------------------------------------------------------ */

@@ -266,8 +266,9 @@ def test_pack_scales_and_zeros_placement_and_padding():
     assert (qw.nbytes, scales.nbytes, qz.nbytes) == O.packed_sizes(N, K)
     for n in range(Np):
         for g in range(G):
-            got_s = scales[g * Np + n]
-            got_z = (qz[g * (Np // 8) + n // 8] >> (4 * (n % 8))) & 0xF
+            unit = (n // 32) * G + g        # unit-major, as the header describes
+            got_s = scales[unit * 32 + n % 32]
+            got_z = (qz[unit * 4 + (n % 32) // 8] >> (4 * (n % 8))) & 0xF
             if n < N:
                 assert got_s == sc[n, g] and got_z == z[n, g]
             else:

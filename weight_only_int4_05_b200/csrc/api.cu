@@ -25,7 +25,7 @@ int num_sms() {
   return cached[dev];
 }
 
-static unsigned* device_status_ptr() {
+unsigned* device_status_ptr() {
   static unsigned* cached[64] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
@@ -127,7 +127,9 @@ awq_status w4a16_gemv(const uint16_t* d_x, const uint32_t* d_qweight, const uint
   awq_status st = check_linear(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g);
   if (st != AWQ_OK) return st;
   if (d_workspace && !aligned16(d_workspace)) return AWQ_ERR_MISALIGNED;
-  return gemv_launch(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, d_workspace, workspace_bytes,
+  unsigned* status = device_status_ptr();
+  if (status == nullptr) return AWQ_ERR_CUDA;
+  return gemv_launch(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, d_workspace, workspace_bytes, status,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -47,15 +47,12 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+// Arrivals discard the returned barrier state (sink operand), so the thread does not wait for it.
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
-  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
-                   smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   unsigned ok;
@@ -97,6 +94,18 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
       "[%4];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+// Fire-and-forget prefetch of `bytes` (multiple of 16, 16-B aligned) of global memory into L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+// 3-D tiled tensor copy global -> shared.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
@@ -172,6 +181,11 @@ __host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);     // M / 16
 }
 
+// Barrier over a subset of the CTA's warps (ids 1..15; `threads` a multiple of 32).
+__device__ __forceinline__ void named_barrier_sync(unsigned id, unsigned threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // ---------------------------------------------------------------- loads
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {  // read-once data: skip L1
   uint4 v;
@@ -181,33 +195,26 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {  // read-once data:
   return v;
 }
 __device__ __forceinline__ uint4 ldg_cached(const void* p) {  // reused data (activations): keep in L1
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
+  return *reinterpret_cast<const uint4*>(p);  // plain load: the compiler folds offsets into the address
 }
 
 // ---------------------------------------------------------------- int4 -> fp16 pairs
-// lop3 with (a & b) | c.  With c = 0x64006400 (fp16 1024 in both halves) and a nibble mask in the
-// low mantissa bits, each 16-bit half becomes the fp16 value 1024 + code (mask 0x000F000F) or
-// 1024 + 16 * code (mask 0x00F000F0), exactly (the bit trick for int4 -> fp16 described by Kim et
-// al., "Who Says Elephants Can't Run", 2022).
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
+// (w & mask) | 0x64006400 puts fp16 1024 in both 16-bit halves with the nibble in the low mantissa
+// bits: each half becomes exactly 1024 + code (mask 0x000F000F) or 1024 + 16 * code (mask 0x00F000F0)
+// -- the bit trick for int4 -> fp16 described by Kim et al., "Who Says Elephants Can't Run", 2022.
+// Written as plain C++ so that the compiler fuses the and/or into one logic op with immediates.
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
 // The four (code - zero) half2 pairs of one packed word, channel order (0,1) (2,3) (4,5) (6,7).
 // z1024 = fp16 (1024 + z) and nz64 = fp16 -(64 + z), each in both halves.  All results are exact.
 __device__ __forceinline__ void word_minus_zero(uint32_t w, __half2 z1024, __half2 nz64, __half2 (&d)[4]) {
-  const __half2 sixteenth = __floats2half2_rn(0.0625f, 0.0625f);
+  const __half2 sixteenth = u32_as_h2(0x2C002C00u);  // fp16 0.0625 in both halves
   const uint32_t t = w >> 8;
-  d[0] = __hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, 0x64006400u)), z1024);
-  d[1] = __hfma2(u32_as_h2(lop3_and_or(w, 0x00F000F0u, 0x64006400u)), sixteenth, nz64);
-  d[2] = __hsub2(u32_as_h2(lop3_and_or(t, 0x000F000Fu, 0x64006400u)), z1024);
-  d[3] = __hfma2(u32_as_h2(lop3_and_or(t, 0x00F000F0u, 0x64006400u)), sixteenth, nz64);
+  d[0] = __hsub2(u32_as_h2((w & 0x000F000Fu) | 0x64006400u), z1024);
+  d[1] = __hfma2(u32_as_h2((w & 0x00F000F0u) | 0x64006400u), sixteenth, nz64);
+  d[2] = __hsub2(u32_as_h2((t & 0x000F000Fu) | 0x64006400u), z1024);
+  d[3] = __hfma2(u32_as_h2((t & 0x00F000F0u) | 0x64006400u), sixteenth, nz64);
 }
 // fp16 (1024 + z) and -(64 + z), splatted into both halves, from a zero point 0..15.
 __device__ __forceinline__ __half2 zero_1024(uint32_t z) { return u32_as_h2((0x6400u | z) * 0x00010001u); }

@@ -4,16 +4,18 @@
 // Weights are the UMMA A operand (M = 128 rows of N), activations the B operand (N = BT tokens), so a
 // small token count still maps onto a full-height MMA.
 //
-// Per CTA (192 threads, one output tile, k-blocks of 64 channels through an ST-stage ring):
-//   warp 0, lane 0  producer: TMA bulk copies of the packed tile (4 row blocks x 1 KB), its fp16 scales
-//                   and packed zeros, and a 2-D tensor copy of the x' tile in the 128-byte swizzle
+// Per CTA (64 + 128 * kDequantWG threads, one output tile, k-blocks of 64 channels through an ST-stage ring):
+//   warp 0, lane 0  producer: four TMA tensor copies per stage -- the codes of the tile's 4 row blocks, their
+//                   fp16 scales and their packed zeros, and a 2-D tensor copy of the x' tile in the 128-byte swizzle
 //                   layout; all complete on full[s].  Weight copies for the first ring are issued before
 //                   griddepcontrol.wait, so they overlap the previous kernel on the stream.
-//   warps 2..5      dequant: thread r owns weight row r of the tile; it turns 64 packed codes into
+//   warps 2..       kDequantWG dequant warpgroups take alternate k-blocks, so one warpgroup's latency
+//                   overlaps the other's.  Thread r of a warpgroup owns weight row r of the tile; it turns 64 packed codes into
 //                   fp16 (q - z) * S (exact q - z by the int4->fp16 bit trick, one rounding for the
 //                   scale) and writes them in the 128-byte swizzle K-major layout the MMA reads, then
 //                   fence.proxy.async + arrive on afull[s].  After the main loop the same warps are
-//                   the epilogue: tcgen05.ld of their 32-lane TMEM quarter, fp16 convert, store y.
+//                   the epilogue (the warpgroups split the columns): tcgen05.ld of their 32-lane TMEM
+//                   quarter, fp16 convert, store y.
 //   warp 1          allocates TMEM (fp32 accumulator, BT columns); lane 0 issues 4 x
 //                   tcgen05.mma.kind::f16 (128 x BT x 16) per k-block and tcgen05.commit -> empty[s].
 // Every mbarrier wait is bounded (see common.cuh); a timeout is recorded in the status word, the CTA
@@ -25,7 +27,11 @@ namespace awq {
 
 constexpr int kBN = 128;  // weight rows per tile (UMMA M)
 constexpr int kBK = 64;   // channels per k-block (one 128-byte swizzle row of fp16)
-constexpr int kGemmThreads = 192;
+#ifndef AWQ_GEMM_DEQUANT_WG
+#define AWQ_GEMM_DEQUANT_WG 2
+#endif
+constexpr int kDequantWG = AWQ_GEMM_DEQUANT_WG;            // dequant warpgroups, alternating k-blocks
+constexpr int kGemmThreads = 64 + 128 * kDequantWG;
 constexpr int kMaxSmem = 232448;  // opt-in dynamic shared memory per block on sm_100
 
 // byte offsets inside one pipeline stage
@@ -42,53 +48,61 @@ struct GemmParams {
   const uint32_t* qzeros;
   uint16_t* y;
   unsigned* status;
+  float* ws_part;    // split-K partial tiles [tile][split][BT][128] fp32 (splits > 1 only)
+  unsigned* ws_cnt;  // per-tile arrival counters (zero between calls)
   int M, N, Np, K, KB, BT, ST, tmem_cols;
+  int splits, kb_per_split;  // k-blocks [split * kb_per_split, ...) per CTA
   uint32_t idesc;
 };
 
-__device__ __forceinline__ void gemm_producer(const CUtensorMap* xmap, const GemmParams& p, uint8_t* smem,
+// Producer (lane 0 of warp 0).  Four TMA copies per stage: a 3-D box of the codes of the tile's 4 row
+// blocks (2 chunks of 512 B each), 2-D boxes of their scales (4 x 64 B) and zeros (4 x 16 B), and the
+// x' tile in the 128-byte swizzle layout.  Row blocks past the end of the weight come back zero-filled.
+struct GemmMaps {
+  CUtensorMap x, codes, scales, zeros;
+};
+
+__device__ __forceinline__ void gemm_producer(const GemmMaps* maps, const GemmParams& p, uint8_t* smem,
                                               uint64_t* full, uint64_t* empty, volatile int* abort_flag,
-                                              int n0, int t0, int rb_avail) {
-  const unsigned pk_bytes = 1024u * rb_avail, sc_bytes = 64u * rb_avail, z_bytes = 16u * rb_avail;
-  const unsigned tx = (unsigned)p.BT * 128u + pk_bytes + sc_bytes + z_bytes;
-  const int KC = p.K / 32;
-  auto issue_w = [&](int kb, int s) {
+                                              int n0, int t0, int kb0, int nkb) {
+  const unsigned tx = (unsigned)p.BT * 128u + 4096u + 256u + 64u;
+  const int rb0 = n0 / 32;
+  auto issue_w = [&](int kk, int s) {  // kk: k-block index within this CTA's range
+    const int kb = kb0 + kk, g = kb >> 1;
     uint8_t* st = smem + (size_t)s * stage_bytes(p.BT);
     mbar_arrive_expect_tx(&full[s], tx);
-    for (int i = 0; i < rb_avail; ++i)
-      bulk_g2s(st + off_pk(p.BT) + i * 1024, p.qw + ((size_t)(n0 / 32 + i) * KC + kb * 2) * 32, 1024u, &full[s]);
-    const int g = kb >> 1;
-    bulk_g2s(st + off_sc(p.BT), p.scales + (size_t)g * p.Np + n0, sc_bytes, &full[s]);
-    bulk_g2s(st + off_z(p.BT), p.qzeros + (size_t)g * (p.Np / 8) + n0 / 8, z_bytes, &full[s]);
+    tma_load_3d(st + off_pk(p.BT), &maps->codes, 0, kb * 2, rb0, &full[s]);
+    tma_load_2d(st + off_sc(p.BT), &maps->scales, g * 32, rb0, &full[s]);
+    tma_load_2d(st + off_z(p.BT), &maps->zeros, g * 4, rb0, &full[s]);
   };
-  auto issue_x = [&](int kb, int s) {
-    tma_load_2d(smem + (size_t)s * stage_bytes(p.BT) + kOffB, xmap, kb * kBK, t0, &full[s]);
+  auto issue_x = [&](int kk, int s) {
+    tma_load_2d(smem + (size_t)s * stage_bytes(p.BT) + kOffB, &maps->x, (kb0 + kk) * kBK, t0, &full[s]);
   };
-  const int pre = p.KB < p.ST ? p.KB : p.ST;
-  for (int kb = 0; kb < pre; ++kb) issue_w(kb, kb);
+  const int pre = nkb < p.ST ? nkb : p.ST;
+  for (int kk = 0; kk < pre; ++kk) issue_w(kk, kk);
   pdl_wait_prior_grids();
-  for (int kb = 0; kb < pre; ++kb) issue_x(kb, kb);
+  for (int kk = 0; kk < pre; ++kk) issue_x(kk, kk);
   int issued = pre;
-  for (int kb = pre; kb < p.KB; ++kb) {
-    const int s = kb % p.ST, use = kb / p.ST;
+  for (int kk = pre; kk < nkb; ++kk) {
+    const int s = kk % p.ST, use = kk / p.ST;
     if (*abort_flag || !mbar_wait(&empty[s], (use - 1) & 1, p.status)) {
       *abort_flag = 1;
       break;
     }
-    issue_w(kb, s);
-    issue_x(kb, s);
-    issued = kb + 1;
+    issue_w(kk, s);
+    issue_x(kk, s);
+    issued = kk + 1;
   }
   if (*abort_flag) {  // wait (bounded) until every copy this thread issued has landed
-    for (int kb = issued > p.ST ? issued - p.ST : 0; kb < issued; ++kb)
-      mbar_wait(&full[kb % p.ST], (kb / p.ST) & 1, p.status);
+    for (int kk = issued > p.ST ? issued - p.ST : 0; kk < issued; ++kk)
+      mbar_wait(&full[kk % p.ST], (kk / p.ST) & 1, p.status);
   }
 }
 
 __device__ __forceinline__ void gemm_mma(const GemmParams& p, uint8_t* smem, uint64_t* full, uint64_t* afull,
                                          uint64_t* empty, uint64_t* accf, volatile int* abort_flag,
-                                         uint32_t tmem) {
-  for (int kb = 0; kb < p.KB; ++kb) {
+                                         uint32_t tmem, int nkb) {
+  for (int kb = 0; kb < nkb; ++kb) {
     const int s = kb % p.ST;
     const unsigned par = (kb / p.ST) & 1;
     if (*abort_flag || !mbar_wait(&full[s], par, p.status) || !mbar_wait(&afull[s], par, p.status)) {
@@ -110,11 +124,11 @@ __device__ __forceinline__ void gemm_mma(const GemmParams& p, uint8_t* smem, uin
 __device__ __forceinline__ void gemm_dequant_epilogue(const GemmParams& p, uint8_t* smem, uint64_t* full,
                                                       uint64_t* afull, uint64_t* accf, volatile int* abort_flag,
                                                       uint32_t tmem, int n0, int t0, int rb_avail, int r,
-                                                      int warp, int lane) {
+                                                      int wg, int warp, int lane, int nkb) {
   const int rbl = r >> 5, rr = r & 31;
   const bool row_ok = rbl < rb_avail;
   const uint32_t swz = (uint32_t)(r & 7);
-  for (int kb = 0; kb < p.KB; ++kb) {
+  for (int kb = wg; kb < nkb; kb += kDequantWG) {  // this warpgroup's k-blocks
     const int s = kb % p.ST;
     if (*abort_flag || !mbar_wait(&full[s], (kb / p.ST) & 1, p.status)) {
       *abort_flag = 1;
@@ -149,36 +163,77 @@ __device__ __forceinline__ void gemm_dequant_epilogue(const GemmParams& p, uint8
 #pragma unroll
       for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(arow + (c << 4)) = make_uint4(0u, 0u, 0u, 0u);
     }
-    fence_proxy_async_smem();
-    mbar_arrive(&afull[s]);
+    fence_proxy_async_smem();  // this thread's generic writes -> visible to the MMA (async proxy)
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&afull[s]);  // one arrival per warp
   }
 
   // ---- epilogue: TMEM lanes 32*q .. 32*q+31 hold weight rows 32*q + lane of the tile
   pdl_wait_prior_grids();
-  const bool acc_ok = mbar_wait(accf, 0, p.status);
+  if (!mbar_wait(accf, 0, p.status)) *abort_flag = 1;
   tc_fence_after_sync();
-  // tcgen05.ld is warp-collective: the whole warp takes the same decision
-  if (!__all_sync(0xFFFFFFFFu, acc_ok && !*abort_flag)) {
-    *abort_flag = 1;
+  // Every epilogue thread reaches this barrier (its wait is bounded); after it the abort flag is final
+  // (the producer and MMA roles are done), so all epilogue warps take the same decision.
+  named_barrier_sync(1, 128 * kDequantWG);
+  if (*abort_flag) return;
+  const int q = warp & 3;
+  const int row = 32 * q + lane;
+  const int n = n0 + row;
+  const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+  if (p.splits == 1) {
+    for (int c0 = 16 * wg; c0 < p.BT; c0 += 16 * kDequantWG) {  // warpgroups split the columns
+      uint32_t v[16];
+      tmem_ld_32x32b_x16(tq + (uint32_t)c0, v);
+      tmem_wait_ld();
+      if (n < p.N) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int t = t0 + c0 + i;
+          if (t < p.M) p.y[(size_t)t * p.N + n] = __half_as_ushort(__float2half_rn(__uint_as_float(v[i])));
+        }
+      }
+    }
     return;
   }
-  const int q = warp & 3;
-  const int n = n0 + 32 * q + lane;
-  for (int c0 = 0; c0 < p.BT; c0 += 16) {
+  // ---- split-K: fp32 partial tile to the workspace; the last split to arrive sums them in order
+  const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+  float* tile_ws = p.ws_part + (size_t)tile * p.splits * p.BT * 128;
+  float* mine = tile_ws + (size_t)blockIdx.z * p.BT * 128;  // [column][row]
+  for (int c0 = 16 * wg; c0 < p.BT; c0 += 16 * kDequantWG) {
     uint32_t v[16];
-    tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+    tmem_ld_32x32b_x16(tq + (uint32_t)c0, v);
     tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mine[(size_t)(c0 + i) * 128 + row] = __uint_as_float(v[i]);
+  }
+  __threadfence();
+  named_barrier_sync(1, 128 * kDequantWG);
+  volatile unsigned* s_last = reinterpret_cast<volatile unsigned*>(abort_flag) + 1;
+  if (threadIdx.x == 64) *s_last = atomicAdd(&p.ws_cnt[tile], 1u) == (unsigned)(p.splits - 1);
+  named_barrier_sync(1, 128 * kDequantWG);
+  if (!*s_last) return;
+  __threadfence();
+  for (int c0 = 16 * wg; c0 < p.BT; c0 += 16 * kDequantWG) {
+    float acc[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+    for (int sp = 0; sp < p.splits; ++sp) {
+      const float* src = tile_ws + (size_t)sp * p.BT * 128;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] += __ldcg(src + (size_t)(c0 + i) * 128 + row);
+    }
     if (n < p.N) {
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int t = t0 + c0 + i;
-        if (t < p.M) p.y[(size_t)t * p.N + n] = __half_as_ushort(__float2half_rn(__uint_as_float(v[i])));
+        if (t < p.M) p.y[(size_t)t * p.N + n] = __half_as_ushort(__float2half_rn(acc[i]));
       }
     }
   }
+  if (threadIdx.x == 64) p.ws_cnt[tile] = 0u;
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap xmap,
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmMaps maps,
                                                                const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -193,17 +248,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kBN, t0 = blockIdx.y * p.BT;
   const int rb_avail = min(4, (p.Np - n0) / 32);
+  const int kb0 = blockIdx.z * p.kb_per_split;
+  const int nkb = min(p.kb_per_split, p.KB - kb0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.ST; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&afull[s], 128);
+      mbar_init(&afull[s], 4);  // the 4 warps of the dequant warpgroup that owns the stage
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    prefetch_tensormap(&xmap);
+    prefetch_tensormap(&maps.x);
+    prefetch_tensormap(&maps.codes);
+    prefetch_tensormap(&maps.scales);
+    prefetch_tensormap(&maps.zeros);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, (unsigned)p.tmem_cols);
@@ -216,12 +276,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   pdl_launch_dependents();
 
   if (warp == 0) {
-    if (lane == 0) gemm_producer(&xmap, p, smem, full, empty, abort_flag, n0, t0, rb_avail);
+    if (lane == 0) gemm_producer(&maps, p, smem, full, empty, abort_flag, n0, t0, kb0, nkb);
   } else if (warp == 1) {
-    if (lane == 0) gemm_mma(p, smem, full, afull, empty, accf, abort_flag, tmem);
+    if (lane == 0) gemm_mma(p, smem, full, afull, empty, accf, abort_flag, tmem, nkb);
   } else {
-    gemm_dequant_epilogue(p, smem, full, afull, accf, abort_flag, tmem, n0, t0, rb_avail, threadIdx.x - 64, warp,
-                          lane);
+    const int wg = (threadIdx.x - 64) >> 7;
+    gemm_dequant_epilogue(p, smem, full, afull, accf, abort_flag, tmem, n0, t0, rb_avail, (threadIdx.x - 64) & 127, wg,
+                          warp, lane, nkb);
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -276,10 +337,38 @@ bool smem_attr_set(int smem) {
 
 }  // namespace
 
-size_t gemm_workspace_bytes(int, int, int) { return 0; }
+struct GemmPlan {
+  int BT, n_tiles, t_tiles, KB, splits, kb_per_split;
+  size_t part_bytes;
+};
+
+// Split K when the output tiles alone cannot occupy the SMs: as many splits as fit in one wave, each
+// with at least 4 k-blocks.
+GemmPlan plan_gemm(int M, int N, int K) {
+  GemmPlan g{};
+  g.BT = pick_bt(M);
+  g.n_tiles = ((N + 31) / 32 * 32 + kBN - 1) / kBN;
+  g.t_tiles = (M + g.BT - 1) / g.BT;
+  g.KB = K / kBK;
+  const int tiles = g.n_tiles * g.t_tiles;
+  int s = tiles >= num_sms() ? 1 : num_sms() / tiles;
+  const int max_by_k = g.KB / 4 > 0 ? g.KB / 4 : 1;
+  if (s > max_by_k) s = max_by_k;
+  if (s < 1) s = 1;
+  g.kb_per_split = (g.KB + s - 1) / s;
+  g.splits = (g.KB + g.kb_per_split - 1) / g.kb_per_split;  // no empty split
+  g.part_bytes = g.splits > 1 ? (size_t)tiles * g.splits * g.BT * 128 * sizeof(float) : 0;
+  return g;
+}
+
+size_t gemm_workspace_bytes(int M, int N, int K) {
+  const GemmPlan g = plan_gemm(M, N, K);
+  return g.part_bytes == 0 ? 0 : kWorkspaceCounterBytes + g.part_bytes;
+}
 
 awq_status gemm_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
-                       uint16_t* y, int M, int N, int K, void*, size_t, unsigned* dev_status, cudaStream_t st) {
+                       uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,
+                       cudaStream_t st) {
   EncodeTiledFn encode = encode_fn();
   if (encode == nullptr) return AWQ_ERR_CUDA;
   GemmParams p;
@@ -293,7 +382,15 @@ awq_status gemm_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
   p.Np = (N + 31) / 32 * 32;
   p.K = K;
   p.KB = K / kBK;
-  p.BT = pick_bt(M);
+  const GemmPlan g = plan_gemm(M, N, K);
+  if ((size_t)g.n_tiles * g.t_tiles * 4 > kWorkspaceCounterBytes) return AWQ_ERR_UNSUPPORTED;
+  if (g.part_bytes > 0 && (ws == nullptr || ws_bytes < kWorkspaceCounterBytes + g.part_bytes))
+    return AWQ_ERR_WORKSPACE;
+  p.ws_cnt = static_cast<unsigned*>(ws);
+  p.ws_part = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWorkspaceCounterBytes) : nullptr;
+  p.splits = g.splits;
+  p.kb_per_split = g.kb_per_split;
+  p.BT = g.BT;
   const int sb = stage_bytes(p.BT);
   p.ST = (kMaxSmem - 2048) / sb;
   if (p.ST > 8) p.ST = 8;
@@ -302,17 +399,47 @@ awq_status gemm_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
   const int smem = p.ST * sb + 1024 + 256;
   if (!smem_attr_set(smem)) return AWQ_ERR_CUDA;
 
-  CUtensorMap xmap;
-  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)p.BT};
-  const cuuint32_t estr[2] = {1, 1};
-  if (encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return AWQ_ERR_CUDA;
-  const dim3 grid((unsigned)((p.Np + kBN - 1) / kBN), (unsigned)((M + p.BT - 1) / p.BT));
-  cudaError_t e = launch_pdl(gemm_kernel, grid, dim3(kGemmThreads), (size_t)smem, st, xmap, p);
+  GemmMaps maps;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint64_t RB = (cuuint64_t)p.Np / 32, G = (cuuint64_t)K / 128;
+  {  // x' [M][K] fp16, 64 x BT boxes in the 128-byte swizzle layout
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)p.BT};
+    if (encode(&maps.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return AWQ_ERR_CUDA;
+  }
+  {  // codes: [RB][K/32 chunks][128 words]; box = 2 chunks x 4 row blocks
+    const cuuint64_t dims[3] = {128, (cuuint64_t)K / 32, RB};
+    const cuuint64_t strides[2] = {512, (cuuint64_t)K / 32 * 512};
+    const cuuint32_t box[3] = {128, 2, 4};
+    if (encode(&maps.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(qw), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return AWQ_ERR_CUDA;
+  }
+  {  // scales: [RB][G * 32] fp16; box = 32 x 4 row blocks
+    const cuuint64_t dims[2] = {G * 32, RB};
+    const cuuint64_t strides[1] = {G * 64};
+    const cuuint32_t box[2] = {32, 4};
+    if (encode(&maps.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(scales), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return AWQ_ERR_CUDA;
+  }
+  {  // zeros: [RB][G * 4] u32; box = 4 x 4 row blocks
+    const cuuint64_t dims[2] = {G * 4, RB};
+    const cuuint64_t strides[1] = {G * 16};
+    const cuuint32_t box[2] = {4, 4};
+    if (encode(&maps.zeros, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(qzeros), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return AWQ_ERR_CUDA;
+  }
+  const dim3 grid((unsigned)g.n_tiles, (unsigned)g.t_tiles, (unsigned)g.splits);
+  cudaError_t e = launch_pdl(gemm_kernel, grid, dim3(kGemmThreads), (size_t)smem, st, maps, p);
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 

@@ -2,27 +2,35 @@
 //
 // y[m][n] = sum_g S[n][g] * sum_{k in g} (q[n][k] - z[n][g]) * x'[m][k]   for up to MT rows of x' per pass.
 //
-// Work decomposition.  The packed layout stores each (32-row block rb, 128-channel group g) as 2048
-// contiguous bytes, so a "unit" u = rb * G + g is one 2 KB stretch of memory and the whole weight is
-// U = (N_pad / 32) * G consecutive units.  T warps share them evenly: warp t owns units
-// [U*t/T, U*(t+1)/T) -- one contiguous range, so every SM streams the same number of bytes and the
-// kernel has no wave-quantization tail.  Inside a warp, lane r owns row 32*rb + r: each unit is four
-// coalesced 128-bit loads per lane (512 contiguous bytes per warp-instruction), dequantized in
-// registers with the int4->fp16 bit trick, multiplied with x' in packed half2 FMAs (partials of 16
-// products, flushed to fp32 every 32 channels), scaled by the group's fp16 scale and accumulated in
-// fp32.  No cross-lane reduction is needed because the layout gives each lane a whole row.
+// Units.  The packed layout stores each (32-row block rb, 128-channel group g) as 2048 contiguous
+// bytes, so unit u = rb * G + g is one 2 KB stretch and the weight is U = RB * G consecutive units.
+// Each of the P CTAs owns a balanced contiguous range (q = U / P units, one more for the first U % P
+// CTAs); its 8 warps split that range into 8 balanced contiguous sub-ranges.  Inside a warp, lane r owns row 32*rb + r: a unit is four
+// coalesced 128-bit loads per lane (512 contiguous bytes per warp-instruction), dequantized in registers
+// with the int4->fp16 bit trick, multiplied with x' in packed half2 FMAs (two independent accumulators,
+// 16 products each, flushed to fp32 every 64 channels), scaled by the group's fp16 scale and
+// accumulated in fp32.  No cross-lane reduction is needed: the layout gives each lane a whole row.
 //
-// Split-K combine.  A row block whose G units are spread over several warps gets one fp32 partial per
-// warp in the workspace slot (rb, t - first_warp(rb)); the warp that brings the per-row-block counter
-// to its final value sums the slots in slot order (deterministic) and writes fp16 y, then resets the
-// counter to 0 for the next call.  Row blocks owned entirely by one warp are written directly.
+// Streaming.  Each warp owns a contiguous sub-range and streams its codes through its own
+// shared-memory ring of kRing 2 KB unit slots with TMA bulk copies, so the bytes in flight cost no
+// registers; the lanes read each unit's scales and zeros themselves, one unit ahead.  Four 8-warp CTAs
+// per SM keep 32 warps issuing.  Before
+// griddepcontrol.wait a kernel touches only its weights -- every warp issues one bulk L2 prefetch of its
+// whole sub-range and fills its ring -- so with programmatic dependent launch the weight stream of the
+// next kernel on the stream starts while this one drains.
 //
-// Programmatic dependent launch: the first unit's weights are loaded before griddepcontrol.wait, so
-// the weight stream of this kernel overlaps the tail of the kernel before it on the stream.
+// Combining split row blocks.  A row block wholly inside one warp's sub-range is written directly.  A
+// row block split between warps of one CTA is summed in shared memory, in warp order.  A row block
+// split between CTAs gets one fp32 partial per CTA in the workspace slot (rb, c - first_cta(rb)); the
+// CTA that brings the row block's counter to its final value sums the slots in slot order
+// (deterministic), writes fp16 y and resets the counter to 0 for the next call.
 #include "common.cuh"
 #include "internal.h"
 
 namespace awq {
+
+constexpr int kGemvThreads = 256;
+constexpr int kGemvWarps = kGemvThreads / 32;
 
 struct GemvParams {
   const uint16_t* x;
@@ -32,183 +40,304 @@ struct GemvParams {
   uint16_t* y;
   float* ws_part;
   unsigned* ws_cnt;
-  long long U;   // units = RB * G
-  long long T;   // warps sharing the units
+  unsigned* status;  // device status word (bounded waits)
+  int U;   // units = RB * G
+  int P;   // CTAs sharing the units: CTA c owns q units, plus one more if c < r
+  int q, r;
   int M, N, Np, K, G, RB, S, m0;
 };
 
-__device__ __forceinline__ long long warp_of_unit(long long u, long long U, long long T) {
-  return ((u + 1) * T - 1) / U;
+__device__ __forceinline__ int cta_first_unit(const GemvParams& p, int c) { return p.q * c + min(c, p.r); }
+__device__ __forceinline__ int cta_of_unit(const GemvParams& p, int u) {
+  const int b = p.r * (p.q + 1);
+  return u < b ? u / (p.q + 1) : p.r + (u - b) / p.q;
 }
 
-__device__ __forceinline__ void load_unit(uint4 (&w)[4], const uint4* qw, long long u, int lane) {
-  const uint4* p = qw + u * 128 + lane;  // unit u = 2048 B = 128 x 16 B; chunk c at +32*c
-#pragma unroll
-  for (int c = 0; c < 4; ++c) w[c] = ldg_stream(p + 32 * c);
+// One shared-memory ring slot per unit: its 2048 B of codes (one TMA bulk copy).  The unit's 64 B of
+// scales and 16 B of zeros are read by the lanes themselves, one unit ahead.
+constexpr int kSlotBytes = 2048;
+constexpr int kSlotStride = 2048;
+#ifndef AWQ_GEMV_RING
+#define AWQ_GEMV_RING 2
+#endif
+constexpr int kRing = AWQ_GEMV_RING;  // units in flight per warp
+constexpr int kRingBytes = kGemvWarps * kRing * kSlotStride;
+
+// Copies the codes of unit u into a ring slot; completion is counted on `bar`.
+__device__ __forceinline__ void issue_unit(const GemvParams& p, int u, uint8_t* slot, uint64_t* bar) {
+  mbar_arrive_expect_tx(bar, kSlotBytes);
+  bulk_g2s(slot, p.qw + (size_t)u * 128, 2048u, bar);
+}
+
+// Scale (as float) and zero point of this lane's row in unit u (coalesced across the warp).
+__device__ __forceinline__ void load_meta(const GemvParams& p, int u, int lane, float& sc, uint32_t& z) {
+  sc = __half2float(p.scales[(size_t)u * 32 + lane]);
+  z = (p.qzeros[(size_t)u * 4 + (lane >> 3)] >> (4 * (lane & 7))) & 0xFu;
 }
 
 template <int MT>
-__global__ void __launch_bounds__(256) gemv_kernel(const GemvParams p) {
-  pdl_launch_dependents();
-  const int lane = threadIdx.x & 31;
-  const long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= p.T) return;  // writes nothing
-  const int mcount = min(MT, p.M - p.m0);
-  long long u = p.U * t / p.T;
-  const long long u_end = p.U * (t + 1) / p.T;
-  const int G = p.G;
-
-  uint4 w[4];
-  load_unit(w, p.qw, u, lane);
-  pdl_wait_prior_grids();  // activations, outputs and workspace belong to the stream order
-
-  // Row pointers of x' for this pass; rows beyond M repeat the last row (computed, never stored).
-  const uint16_t* xrow[MT];
+__device__ __forceinline__ void unit_dot(const uint4 (&w)[4], float sc, uint32_t z,
+                                         const uint16_t* __restrict__ const (&xg)[MT],
+                                         float (&yacc)[MT]) {
+  const __half2 z1024 = zero_1024(z), nz64 = neg_zero_64(z);
+  float part[MT];
 #pragma unroll
-  for (int m = 0; m < MT; ++m) xrow[m] = p.x + (size_t)(p.m0 + min(m, mcount - 1)) * p.K;
-
-  while (u < u_end) {
-    const int rb = (int)(u / G);
-    const int g0 = (int)(u - (long long)rb * G);
-    const long long seg_end = min(u_end, (long long)(rb + 1) * G);
-    const int n = rb * 32 + lane;
-    float yacc[MT];
+  for (int m = 0; m < MT; ++m) part[m] = 0.f;
+#pragma unroll(MT >= 4 ? 1 : 2)
+  for (int cp = 0; cp < 2; ++cp) {  // pairs of 32-channel chunks
+    __half2 acc[2][MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) yacc[m] = 0.f;
-
-    for (; u < seg_end; ++u) {
-      const int g = (int)(u - (long long)rb * G);
-      uint4 wn[4];
-      const bool more = (u + 1 < u_end);
-      if (more) load_unit(wn, p.qw, u + 1, lane);
-      const float scf = __half2float(p.scales[(size_t)g * p.Np + n]);
-      const uint32_t zw = p.qzeros[(size_t)g * (p.Np >> 3) + rb * 4 + (lane >> 3)];
-      const uint32_t z = (zw >> (4 * (lane & 7))) & 0xFu;
-      const __half2 z1024 = zero_1024(z), nz64 = neg_zero_64(z);
-      float part[MT];
+    for (int m = 0; m < MT; ++m) acc[0][m] = acc[1][m] = u32_as_h2(0u);
 #pragma unroll
-      for (int m = 0; m < MT; ++m) part[m] = 0.f;
+    for (int c2 = 0; c2 < 2; ++c2) {
+      const int c = cp * 2 + c2;
+      const uint32_t ww[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t ww[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
-        __half2 acc[MT];
+      for (int j = 0; j < 4; ++j) {
+        __half2 d[4];
+        word_minus_zero(ww[j], z1024, nz64, d);
+        const int a = j & 1;  // two independent accumulator chains
 #pragma unroll
-        for (int m = 0; m < MT; ++m) acc[m] = __float2half2_rn(0.f);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          __half2 d[4];
-          word_minus_zero(ww[j], z1024, nz64, d);
-#pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            const uint4 xv = ldg_cached(xrow[m] + g * 128 + c * 32 + j * 8);
-            acc[m] = __hfma2(d[0], u32_as_h2(xv.x), acc[m]);
-            acc[m] = __hfma2(d[1], u32_as_h2(xv.y), acc[m]);
-            acc[m] = __hfma2(d[2], u32_as_h2(xv.z), acc[m]);
-            acc[m] = __hfma2(d[3], u32_as_h2(xv.w), acc[m]);
-          }
+        for (int m = 0; m < MT; ++m) {
+          const uint4 xv = ldg_cached(xg[m] + c * 32 + j * 8);
+          acc[a][m] = __hfma2(d[0], u32_as_h2(xv.x), acc[a][m]);
+          acc[a][m] = __hfma2(d[1], u32_as_h2(xv.y), acc[a][m]);
+          acc[a][m] = __hfma2(d[2], u32_as_h2(xv.z), acc[a][m]);
+          acc[a][m] = __hfma2(d[3], u32_as_h2(xv.w), acc[a][m]);
         }
-#pragma unroll
-        for (int m = 0; m < MT; ++m) part[m] += __low2float(acc[m]) + __high2float(acc[m]);
-      }
-#pragma unroll
-      for (int m = 0; m < MT; ++m) yacc[m] = fmaf(scf, part[m], yacc[m]);
-      if (more) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) w[c] = wn[c];
       }
     }
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+      part[m] += (__low2float(acc[0][m]) + __high2float(acc[0][m])) +
+                 (__low2float(acc[1][m]) + __high2float(acc[1][m]));
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) yacc[m] = fmaf(sc, part[m], yacc[m]);
+}
 
-    const bool whole = (g0 == 0) && (seg_end == (long long)(rb + 1) * G);
-    if (whole) {
-      if (n < p.N) {
+template <int MT>
+__device__ __forceinline__ void store_y(const GemvParams& p, int rb, int lane, const float (&v)[MT]) {
+  const int n = rb * 32 + lane;
+  const int mcount = min(MT, p.M - p.m0);
+  if (n < p.N) {
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
-          if (m < mcount) p.y[(size_t)(p.m0 + m) * p.N + n] = __half_as_ushort(__float2half_rn(yacc[m]));
-      }
-      continue;
-    }
-    // ---- split-K combine through the workspace
-    const long long tf = warp_of_unit((long long)rb * G, p.U, p.T);
-    const long long tl = warp_of_unit((long long)rb * G + G - 1, p.U, p.T);
-    const int nc = (int)(tl - tf + 1);
-    const int slot = (int)(t - tf);
-    float* base = p.ws_part + (size_t)rb * p.S * 32 * MT;
-#pragma unroll
-    for (int m = 0; m < MT; ++m) base[(size_t)(slot * MT + m) * 32 + lane] = yacc[m];
-    __threadfence();
-    __syncwarp();
-    unsigned old = 0;
-    if (lane == 0) old = atomicAdd(&p.ws_cnt[rb], 1u);
-    old = __shfl_sync(0xFFFFFFFFu, old, 0);
-    if (old == (unsigned)(nc - 1)) {
-      __threadfence();
-      float sum[MT];
-#pragma unroll
-      for (int m = 0; m < MT; ++m) sum[m] = 0.f;
-      for (int j = 0; j < nc; ++j) {
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-          sum[m] += (j == slot) ? yacc[m] : __ldcg(&base[(size_t)(j * MT + m) * 32 + lane]);
-      }
-      if (n < p.N) {
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-          if (m < mcount) p.y[(size_t)(p.m0 + m) * p.N + n] = __half_as_ushort(__float2half_rn(sum[m]));
-      }
-      if (lane == 0) p.ws_cnt[rb] = 0u;
-    }
+    for (int m = 0; m < MT; ++m)
+      if (m < mcount) p.y[(size_t)(p.m0 + m) * p.N + n] = __half_as_ushort(__float2half_rn(v[m]));
   }
 }
 
-// ------------------------------------------------------------------------------------------ host
-namespace {
+// Sum over the CTAs that share row block r (called by the one warp per CTA that combines r).
+template <int MT>
+__device__ __forceinline__ void cross_cta_combine(const GemvParams& p, int r, int lane, const float (&part)[MT]) {
+  const int cf = cta_of_unit(p, r * p.G);
+  const int cl = cta_of_unit(p, r * p.G + p.G - 1);
+  const int nc = cl - cf + 1;
+  const int slot = (int)blockIdx.x - cf;
+  float* base = p.ws_part + (size_t)r * p.S * 32 * MT;  // slots of row block r
+#pragma unroll
+  for (int m = 0; m < MT; ++m) base[(size_t)(slot * MT + m) * 32 + lane] = part[m];
+  __threadfence();
+  __syncwarp();
+  unsigned old = 0;
+  if (lane == 0) old = atomicAdd(&p.ws_cnt[r], 1u);
+  old = __shfl_sync(0xFFFFFFFFu, old, 0);
+  if (old != (unsigned)(nc - 1)) return;
+  __threadfence();
+  float sum[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) sum[m] = 0.f;
+  for (int j = 0; j < nc; ++j) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) sum[m] += (j == slot) ? part[m] : __ldcg(&base[(size_t)(j * MT + m) * 32 + lane]);
+  }
+  store_y<MT>(p, r, lane, sum);
+  if (lane == 0) p.ws_cnt[r] = 0u;
+}
 
-constexpr int kGemvThreads = 256;
-constexpr int kGemvWarps = kGemvThreads / 32;
+template <int MT>
+__global__ void __launch_bounds__(kGemvThreads, (MT == 1 ? 4 : MT == 2 ? 2 : 1)) gemv_kernel(const GemvParams p) {
+  extern __shared__ __align__(128) uint8_t ring_smem[];
+  __shared__ __align__(8) uint64_t full[kGemvWarps][kRing];
+  __shared__ float s_part[kGemvWarps][2][MT * 32];
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = p.G;
+  const int c = blockIdx.x;
+  const int cu0 = cta_first_unit(p, c), n = p.q + (c < p.r ? 1 : 0), cu1 = cu0 + n;
+  const int wq = n >> 3, wr = n & 7;  // kGemvWarps == 8
+  const int wu0 = cu0 + wq * warp + min(warp, wr), nw = wq + (warp < wr ? 1 : 0), wu1 = wu0 + nw;
+  const bool active = nw > 0;
+  uint8_t* ring = ring_smem + (size_t)warp * kRing * kSlotStride;
+
+  // Before the dependency wait: only weights.  The warp's whole sub-range goes towards L2, and the
+  // first kRing units into this warp's shared-memory ring.
+  if (active && lane == 0) {
+#pragma unroll
+    for (int i = 0; i < kRing; ++i) mbar_init(&full[warp][i], 1);
+    fence_mbar_init();
+    const char* base = reinterpret_cast<const char*>(p.qw + (size_t)wu0 * 128);
+    for (int off = 0; off < nw * 2048; off += 32768)
+      prefetch_l2_bulk(base + off, (unsigned)min(32768, nw * 2048 - off));
+    prefetch_l2_bulk(p.scales + (size_t)wu0 * 32, (unsigned)(nw * 64));
+    prefetch_l2_bulk(p.qzeros + (size_t)wu0 * 4, (unsigned)(nw * 16));
+    for (int i = 0; i < kRing && i < nw; ++i) issue_unit(p, wu0 + i, ring + i * kSlotStride, &full[warp][i]);
+  }
+  __syncwarp();
+  pdl_wait_prior_grids();  // activations, outputs and workspace follow the stream order
+
+  const int mcount = min(MT, p.M - p.m0);
+  const uint16_t* xrow[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) xrow[m] = p.x + (size_t)(p.m0 + min(m, mcount - 1)) * p.K;
+  float sc = 0.f;
+  uint32_t z = 0u;
+  if (active) load_meta(p, wu0, lane, sc, z);
+  const int rb_f = active ? wu0 / G : -1;  // the only division of the main path
+  const int g0 = active ? wu0 - rb_f * G : 0;
+
+  bool ok = true;
+  int rb = rb_f, g = g0, rb_l = rb_f;
+  int t = 0;  // units of this warp consumed so far
+  while (t < nw && ok) {  // segments: the units of one row block inside this warp's range
+    const int seg = min(nw - t, G - g);
+    const bool whole = (g == 0) && (seg == G);
+    float yacc[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) yacc[m] = 0.f;
+    for (int i = 0; i < seg; ++i, ++t) {
+      const int si = t & (kRing - 1);
+      uint8_t* slot = ring + si * kSlotStride;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[warp][si], (unsigned)(t / kRing) & 1u, p.status));
+      if (!ok) break;  // warp-uniform
+      float scn = 0.f;
+      uint32_t zn = 0u;
+      if (t + 1 < nw) load_meta(p, wu0 + t + 1, lane, scn, zn);  // next unit's scale and zero
+      uint4 w[4];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) w[cc] = *reinterpret_cast<const uint4*>(slot + cc * 512 + lane * 16);
+      const uint16_t* xg[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) xg[m] = xrow[m] + (g + i) * 128;
+      unit_dot<MT>(w, sc, z, xg, yacc);
+      __syncwarp();  // every lane has consumed the slot
+      if (lane == 0 && t + kRing < nw) {
+        fence_proxy_async_smem();  // our generic reads of the slot before the async-proxy refill
+        issue_unit(p, wu0 + t + kRing, slot, &full[warp][si]);
+      }
+      sc = scn;
+      z = zn;
+    }
+    if (!ok) break;
+    if (whole) {
+      store_y<MT>(p, rb, lane, yacc);
+    } else {
+      const int slot = (rb == rb_f) ? 0 : 1;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) s_part[warp][slot][m * 32 + lane] = yacc[m];
+    }
+    rb_l = rb;
+    ++rb;
+    g = 0;
+  }
+  if (!ok && lane == 0) {  // give up: wait (bounded) for this warp's copies still in flight
+    for (int j = t; j < nw && j < t + kRing; ++j)
+      mbar_wait(&full[warp][j & (kRing - 1)], (unsigned)(j / kRing) & 1u, p.status);
+  }
+  __syncthreads();
+  if (!active || !ok) return;
+
+  // A split row block r is combined by the warp holding its first unit inside this CTA.
+  auto combine = [&](int r) {
+    const int a = max(r * G, cu0), b = min((r + 1) * G, cu1);
+    float sum[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) sum[m] = 0.f;
+    for (int j = warp; j < kGemvWarps; ++j) {
+      const int j0 = cu0 + wq * j + min(j, wr), jn = wq + (j < wr ? 1 : 0);
+      if (j0 >= b) break;
+      if (jn == 0) continue;
+      const int slot = (j0 >= r * G) ? 0 : 1;  // r is warp j's first row block iff it starts at or before j0
+#pragma unroll
+      for (int m = 0; m < MT; ++m) sum[m] += s_part[j][slot][m * 32 + lane];
+    }
+    if (a == r * G && b == (r + 1) * G) store_y<MT>(p, r, lane, sum);
+    else cross_cta_combine<MT>(p, r, lane, sum);
+  };
+  const bool whole_f = (g0 == 0) && (nw >= G);
+  const bool owner_f = (g0 == 0) || (wu0 == cu0);
+  if (owner_f && !whole_f) combine(rb_f);
+  if (rb_l != rb_f && wu1 - rb_l * G < G) combine(rb_l);
+}
+
+// ------------------------------------------------------------------------------------------ host
+#ifndef AWQ_GEMV_CTAS_PER_SM
+#define AWQ_GEMV_CTAS_PER_SM 4
+#endif
+#ifndef AWQ_GEMV_WHOLE_RB_MAX_UNITS
+#define AWQ_GEMV_WHOLE_RB_MAX_UNITS 48
+#endif
+
+namespace {
 
 int pick_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
 template <int MT>
-int gemv_ctas_per_sm() {
+int resident_ctas_mt() {
   static int cached[64] = {0};
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
   if (cached[dev] == 0) {
     int occ = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<MT>, kGemvThreads, 0);
-    cached[dev] = occ > 0 ? occ : 1;
+    cudaFuncSetAttribute(gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingBytes);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<MT>, kGemvThreads, kRingBytes) !=
+            cudaSuccess || occ < 1)
+      occ = 1;
+    cached[dev] = occ < AWQ_GEMV_CTAS_PER_SM ? occ : AWQ_GEMV_CTAS_PER_SM;
   }
   return cached[dev];
 }
 
-int ctas_per_sm(int MT) {
+// CTAs of one GEMV launch per SM: all resident at once (at most AWQ_GEMV_CTAS_PER_SM).
+int resident_ctas(int MT) {
   switch (MT) {
-    case 1: return gemv_ctas_per_sm<1>();
-    case 2: return gemv_ctas_per_sm<2>();
-    case 4: return gemv_ctas_per_sm<4>();
-    default: return gemv_ctas_per_sm<8>();
+    case 1: return resident_ctas_mt<1>();
+    case 2: return resident_ctas_mt<2>();
+    case 4: return resident_ctas_mt<4>();
+    default: return resident_ctas_mt<8>();
   }
 }
 
 struct GemvPlan {
-  int MT, RB, G, S, Np;
-  long long U, T;
+  int MT, RB, G, S, Np, P;
+  int U, q, r;
   size_t part_bytes;
 };
 
+// P CTAs share the U units.  When the row blocks are short (G small) and numerous enough to occupy at
+// least half the SMs, every CTA takes one whole row block, so no partial sum leaves a CTA; otherwise
+// the units are spread evenly over AWQ_GEMV_CTAS_PER_SM CTAs per SM and the row blocks cut by CTA
+// boundaries are combined in the workspace.
 GemvPlan plan_gemv(int M, int N, int K) {
   GemvPlan pl{};
   pl.MT = pick_mt(M);
   pl.Np = (N + 31) / 32 * 32;
   pl.RB = pl.Np / 32;
   pl.G = K / 128;
-  pl.U = (long long)pl.RB * pl.G;
-  const long long slots = (long long)num_sms() * ctas_per_sm(pl.MT) * kGemvWarps;
-  pl.T = pl.U < slots ? pl.U : slots;
-  const long long L = pl.U / pl.T;  // >= 1
-  pl.S = pl.G >= 2 ? (int)((pl.G - 2) / L + 2) : 1;
-  pl.part_bytes = (size_t)pl.RB * pl.S * 32 * pl.MT * sizeof(float);
+  pl.U = pl.RB * pl.G;
+  int p_bal = num_sms() * resident_ctas(pl.MT);
+  const int by_units = pl.U / kGemvWarps > 0 ? pl.U / kGemvWarps : 1;
+  if (p_bal > by_units) p_bal = by_units;
+  if (pl.RB <= p_bal && 2 * pl.RB >= num_sms() && pl.G <= AWQ_GEMV_WHOLE_RB_MAX_UNITS) {
+    pl.P = pl.RB;
+    pl.S = 1;
+    pl.part_bytes = 0;
+  } else {
+    pl.P = p_bal;
+    const int L = pl.U / pl.P;  // >= 1 units per CTA
+    pl.S = pl.G >= 2 ? (pl.G - 2) / L + 2 : 1;
+    pl.part_bytes = (size_t)pl.RB * pl.S * 32 * pl.MT * sizeof(float);
+  }
   return pl;
 }
 
@@ -216,14 +345,36 @@ GemvPlan plan_gemv(int M, int N, int K) {
 
 size_t gemv_workspace_bytes(int M, int N, int K) {
   const GemvPlan pl = plan_gemv(M, N, K);
-  return kWorkspaceCounterBytes + pl.part_bytes;
+  return pl.part_bytes == 0 ? 0 : kWorkspaceCounterBytes + pl.part_bytes;
+}
+
+template <int MT>
+bool gemv_smem_attr() {
+  static bool done[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingBytes) !=
+        cudaSuccess)
+      return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
+template <int MT>
+cudaError_t launch_mt(const GemvParams& p, cudaStream_t st) {
+  if (!gemv_smem_attr<MT>()) return cudaErrorInvalidValue;
+  return launch_pdl(gemv_kernel<MT>, dim3((unsigned)p.P), dim3(kGemvThreads), (size_t)kRingBytes, st, p);
 }
 
 awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
-                       uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, cudaStream_t st) {
+                       uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,
+                       cudaStream_t st) {
   const GemvPlan pl = plan_gemv(M, N, K);
-  if (pl.RB * 4 > (int)(kWorkspaceCounterBytes)) return AWQ_ERR_UNSUPPORTED;
-  if (ws == nullptr || ws_bytes < kWorkspaceCounterBytes + pl.part_bytes) return AWQ_ERR_WORKSPACE;
+  if ((size_t)pl.RB * 4 > kWorkspaceCounterBytes) return AWQ_ERR_UNSUPPORTED;
+  if (pl.part_bytes > 0 && (ws == nullptr || ws_bytes < kWorkspaceCounterBytes + pl.part_bytes))
+    return AWQ_ERR_WORKSPACE;
   GemvParams p;
   p.x = x;
   p.qw = reinterpret_cast<const uint4*>(qw);
@@ -231,9 +382,11 @@ awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
   p.qzeros = qzeros;
   p.y = y;
   p.ws_cnt = static_cast<unsigned*>(ws);
-  p.ws_part = reinterpret_cast<float*>(static_cast<char*>(ws) + kWorkspaceCounterBytes);
+  p.ws_part = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWorkspaceCounterBytes) : nullptr;
   p.U = pl.U;
-  p.T = pl.T;
+  p.P = pl.P;
+  p.q = pl.U / pl.P;
+  p.r = pl.U % pl.P;
   p.M = M;
   p.N = N;
   p.Np = pl.Np;
@@ -241,16 +394,16 @@ awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
   p.G = pl.G;
   p.RB = pl.RB;
   p.S = pl.S;
-  const unsigned grid = (unsigned)((pl.T + kGemvWarps - 1) / kGemvWarps);
+  p.status = dev_status;
   // passes of MT rows run one after the other on the stream and share the workspace
   for (int m0 = 0; m0 < M; m0 += pl.MT) {
     p.m0 = m0;
     cudaError_t e;
     switch (pl.MT) {
-      case 1: e = launch_pdl(gemv_kernel<1>, dim3(grid), dim3(kGemvThreads), 0, st, p); break;
-      case 2: e = launch_pdl(gemv_kernel<2>, dim3(grid), dim3(kGemvThreads), 0, st, p); break;
-      case 4: e = launch_pdl(gemv_kernel<4>, dim3(grid), dim3(kGemvThreads), 0, st, p); break;
-      default: e = launch_pdl(gemv_kernel<8>, dim3(grid), dim3(kGemvThreads), 0, st, p); break;
+      case 1: e = launch_mt<1>(p, st); break;
+      case 2: e = launch_mt<2>(p, st); break;
+      case 4: e = launch_mt<4>(p, st); break;
+      default: e = launch_mt<8>(p, st); break;
     }
     if (e != cudaSuccess) return AWQ_ERR_CUDA;
   }

@@ -46,7 +46,9 @@ awq_status pack_launch(const uint16_t* W, const uint16_t* s, int N, int K, uint3
                        uint32_t* qz, cudaStream_t st);
 size_t gemv_workspace_bytes(int M, int N, int K);
 awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
-                       uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, cudaStream_t st);
+                       uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,
+                       cudaStream_t st);
+unsigned* device_status_ptr();  // address of the device status word on the current device
 size_t gemm_workspace_bytes(int M, int N, int K);
 awq_status gemm_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
                        uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,

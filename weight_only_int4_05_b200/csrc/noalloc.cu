@@ -45,7 +45,9 @@ extern "C" awq_status w4a16_gemv_noalloc(const uint16_t* d_x, const uint32_t* d_
   if (gemv_workspace_bytes(M, N, K) > kNoAllocScratchBytes) return AWQ_ERR_WORKSPACE;
   void* scratch = noalloc_scratch_address();
   if (scratch == nullptr) return AWQ_ERR_CUDA;
+  unsigned* status = device_status_ptr();
+  if (status == nullptr) return AWQ_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(scratch, 0, kWorkspaceCounterBytes, s) != cudaSuccess) return AWQ_ERR_CUDA;
-  return gemv_launch(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, scratch, kNoAllocScratchBytes, s);
+  return gemv_launch(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, scratch, kNoAllocScratchBytes, status, s);
 }

@@ -11,7 +11,7 @@
 // One CTA per packed unit (32-row block rb, group g): 8 warps x 4 rows, lane l holds channels
 // 4l..4l+3 of the group (one 8-byte load per row), min/max by warp shuffles, codes assembled into the
 // nibble order of the layout with one shuffle, and the 2 KB unit written from shared memory with
-// coalesced 16-byte stores.  The kernel streams 2 bytes in and 0.52 bytes out per weight.
+// coalesced 16-byte stores (the unit's 32 scales and 4 zero words are contiguous too).  The kernel streams 2 bytes in and 0.52 bytes out per weight.
 #include "common.cuh"
 #include "internal.h"
 
@@ -92,12 +92,13 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
   __syncthreads();
   if (threadIdx.x < 128)
     qw[((size_t)rb * G + g) * 128 + threadIdx.x] = reinterpret_cast<const uint4*>(s_words)[threadIdx.x];
-  if (threadIdx.x < 32) scales[(size_t)g * Np + rb * 32 + threadIdx.x] = s_sc[threadIdx.x];
+  const size_t unit = (size_t)rb * G + g;  // scales and zeros are unit major
+  if (threadIdx.x < 32) scales[unit * 32 + threadIdx.x] = s_sc[threadIdx.x];
   if (threadIdx.x < 4) {
     uint32_t zw = 0u;
 #pragma unroll
     for (int i = 0; i < 8; ++i) zw |= s_z[threadIdx.x * 8 + i] << (4 * i);
-    qz[(size_t)g * (Np / 8) + rb * 4 + threadIdx.x] = zw;
+    qz[unit * 4 + threadIdx.x] = zw;
   }
 }
 
