@@ -78,6 +78,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsign
     }
   }
 }
+// The same bounded wait with a short sleep between polls, for warps that share their scheduler with
+// working warps (a poll that fails gives its issue slots back).
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, unsigned parity, unsigned* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (unsigned it = 0;; ++it) {
+    __nanosleep(64);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicExch(status, kDevTimeout);
+      return false;
+    }
+  }
+}
 
 // ---------------------------------------------------------------- TMA (bulk and tensor copies)
 // 1-D bulk copy global -> shared, completion counted on `bar` (bytes and addresses 16-B aligned).
@@ -206,15 +220,32 @@ __device__ __forceinline__ uint4 ldg_cached(const void* p) {  // reused data (ac
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
+// (w & MASK) | magic in one logic instruction: the mask is an immediate, the magic a register.
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t and_or(uint32_t w, uint32_t magic) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "r"(magic));
+  return d;
+}
+// fp16 1024 in both halves, as an opaque register value (so the compiler keeps it in a register
+// instead of rebuilding the constant for every use).
+__device__ __forceinline__ uint32_t magic_1024x2() {
+  uint32_t m;
+  asm volatile("mov.b32 %0, 0x64006400;" : "=r"(m));
+  return m;
+}
+
 // The four (code - zero) half2 pairs of one packed word, channel order (0,1) (2,3) (4,5) (6,7).
-// z1024 = fp16 (1024 + z) and nz64 = fp16 -(64 + z), each in both halves.  All results are exact.
-__device__ __forceinline__ void word_minus_zero(uint32_t w, __half2 z1024, __half2 nz64, __half2 (&d)[4]) {
+// z1024 = fp16 (1024 + z) and nz64 = fp16 -(64 + z), each in both halves; magic = magic_1024x2().
+// All results are exact small integers.
+__device__ __forceinline__ void word_minus_zero(uint32_t w, __half2 z1024, __half2 nz64, uint32_t magic,
+                                                __half2 (&d)[4]) {
   const __half2 sixteenth = u32_as_h2(0x2C002C00u);  // fp16 0.0625 in both halves
   const uint32_t t = w >> 8;
-  d[0] = __hsub2(u32_as_h2((w & 0x000F000Fu) | 0x64006400u), z1024);
-  d[1] = __hfma2(u32_as_h2((w & 0x00F000F0u) | 0x64006400u), sixteenth, nz64);
-  d[2] = __hsub2(u32_as_h2((t & 0x000F000Fu) | 0x64006400u), z1024);
-  d[3] = __hfma2(u32_as_h2((t & 0x00F000F0u) | 0x64006400u), sixteenth, nz64);
+  d[0] = __hsub2(u32_as_h2(and_or<0x000F000Fu>(w, magic)), z1024);
+  d[1] = __hfma2(u32_as_h2(and_or<0x00F000F0u>(w, magic)), sixteenth, nz64);
+  d[2] = __hsub2(u32_as_h2(and_or<0x000F000Fu>(t, magic)), z1024);
+  d[3] = __hfma2(u32_as_h2(and_or<0x00F000F0u>(t, magic)), sixteenth, nz64);
 }
 // fp16 (1024 + z) and -(64 + z), splatted into both halves, from a zero point 0..15.
 __device__ __forceinline__ __half2 zero_1024(uint32_t z) { return u32_as_h2((0x6400u | z) * 0x00010001u); }

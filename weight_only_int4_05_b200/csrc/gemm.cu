@@ -142,6 +142,7 @@ __device__ __forceinline__ void gemm_dequant_epilogue(const GemmParams& p, uint8
       const uint32_t z = (zw >> (4 * (r & 7))) & 0xFu;
       const __half2 sc2 = u32_as_h2((uint32_t)scb * 0x00010001u);
       const __half2 z1024 = zero_1024(z), nz64 = neg_zero_64(z);
+      const uint32_t magic = magic_1024x2();
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const uint4 pk = *reinterpret_cast<const uint4*>(st + off_pk(p.BT) + rbl * 1024 + j * 512 + rr * 16);
@@ -149,7 +150,7 @@ __device__ __forceinline__ void gemm_dequant_epilogue(const GemmParams& p, uint8
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
           __half2 d[4];
-          word_minus_zero(ww[wi], z1024, nz64, d);
+          word_minus_zero(ww[wi], z1024, nz64, magic, d);
           uint4 v;
           v.x = h2_as_u32(__hmul2(d[0], sc2));
           v.y = h2_as_u32(__hmul2(d[1], sc2));

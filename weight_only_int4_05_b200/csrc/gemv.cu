@@ -5,7 +5,7 @@
 // Units.  The packed layout stores each (32-row block rb, 128-channel group g) as 2048 contiguous
 // bytes, so unit u = rb * G + g is one 2 KB stretch and the weight is U = RB * G consecutive units.
 // Each of the P CTAs owns a balanced contiguous range (q = U / P units, one more for the first U % P
-// CTAs); its 8 warps split that range into 8 balanced contiguous sub-ranges.  Inside a warp, lane r owns row 32*rb + r: a unit is four
+// CTAs); its NW warps split that range into NW balanced contiguous sub-ranges.  Inside a warp, lane r owns row 32*rb + r: a unit is four
 // coalesced 128-bit loads per lane (512 contiguous bytes per warp-instruction), dequantized in registers
 // with the int4->fp16 bit trick, multiplied with x' in packed half2 FMAs (two independent accumulators,
 // 16 products each, flushed to fp32 every 64 channels), scaled by the group's fp16 scale and
@@ -29,8 +29,6 @@
 
 namespace awq {
 
-constexpr int kGemvThreads = 256;
-constexpr int kGemvWarps = kGemvThreads / 32;
 
 struct GemvParams {
   const uint16_t* x;
@@ -58,10 +56,12 @@ __device__ __forceinline__ int cta_of_unit(const GemvParams& p, int u) {
 constexpr int kSlotBytes = 2048;
 constexpr int kSlotStride = 2048;
 #ifndef AWQ_GEMV_RING
-#define AWQ_GEMV_RING 2
+#define AWQ_GEMV_RING 4
 #endif
 constexpr int kRing = AWQ_GEMV_RING;  // units in flight per warp
-constexpr int kRingBytes = kGemvWarps * kRing * kSlotStride;
+__host__ __device__ constexpr int ring_bytes(int nw) { return nw * kRing * kSlotStride; }
+// Activations staged in shared memory (one TMA copy per row after the dependency wait) when they fit.
+constexpr int kXsMaxBytes = 32 * 1024;
 
 // Copies the codes of unit u into a ring slot; completion is counted on `bar`.
 __device__ __forceinline__ void issue_unit(const GemvParams& p, int u, uint8_t* slot, uint64_t* bar) {
@@ -80,6 +80,7 @@ __device__ __forceinline__ void unit_dot(const uint4 (&w)[4], float sc, uint32_t
                                          const uint16_t* __restrict__ const (&xg)[MT],
                                          float (&yacc)[MT]) {
   const __half2 z1024 = zero_1024(z), nz64 = neg_zero_64(z);
+  const uint32_t magic = magic_1024x2();
   float part[MT];
 #pragma unroll
   for (int m = 0; m < MT; ++m) part[m] = 0.f;
@@ -95,7 +96,7 @@ __device__ __forceinline__ void unit_dot(const uint4 (&w)[4], float sc, uint32_t
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         __half2 d[4];
-        word_minus_zero(ww[j], z1024, nz64, d);
+        word_minus_zero(ww[j], z1024, nz64, magic, d);
         const int a = j & 1;  // two independent accumulator chains
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
@@ -155,23 +156,32 @@ __device__ __forceinline__ void cross_cta_combine(const GemvParams& p, int r, in
   if (lane == 0) p.ws_cnt[r] = 0u;
 }
 
-template <int MT>
-__global__ void __launch_bounds__(kGemvThreads, (MT == 1 ? 4 : MT == 2 ? 2 : 1)) gemv_kernel(const GemvParams p) {
+// NW warps per CTA: 8, 16 or 32.  A 16-warp CTA takes half an SM (64 registers per thread), so the
+// next kernel's CTAs can already be resident beside it; a 32-warp CTA takes a whole SM.
+template <int MT, int NW, bool XS>
+__global__ void __launch_bounds__(NW * 32, (NW == 32 ? 1 : NW == 16 ? 2 : MT == 1 ? 4 : MT == 2 ? 2 : 1))
+    gemv_kernel(const GemvParams p) {
   extern __shared__ __align__(128) uint8_t ring_smem[];
-  __shared__ __align__(8) uint64_t full[kGemvWarps][kRing];
-  __shared__ float s_part[kGemvWarps][2][MT * 32];
+  __shared__ __align__(8) uint64_t full[NW][kRing];
+  __shared__ __align__(8) uint64_t xbar;
+  __shared__ float s_part[NW][2][MT * 32];
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = p.G;
   const int c = blockIdx.x;
   const int cu0 = cta_first_unit(p, c), n = p.q + (c < p.r ? 1 : 0), cu1 = cu0 + n;
-  const int wq = n >> 3, wr = n & 7;  // kGemvWarps == 8
+  const int wq = n / NW, wr = n % NW;  // NW is a power of two
   const int wu0 = cu0 + wq * warp + min(warp, wr), nw = wq + (warp < wr ? 1 : 0), wu1 = wu0 + nw;
   const bool active = nw > 0;
   uint8_t* ring = ring_smem + (size_t)warp * kRing * kSlotStride;
 
   // Before the dependency wait: only weights.  The warp's whole sub-range goes towards L2, and the
   // first kRing units into this warp's shared-memory ring.
+  if (XS && threadIdx.x == 0) {
+    mbar_init(&xbar, 1);
+    fence_mbar_init();
+  }
+  if (XS) __syncthreads();
   if (active && lane == 0) {
 #pragma unroll
     for (int i = 0; i < kRing; ++i) mbar_init(&full[warp][i], 1);
@@ -184,19 +194,30 @@ __global__ void __launch_bounds__(kGemvThreads, (MT == 1 ? 4 : MT == 2 ? 2 : 1))
     for (int i = 0; i < kRing && i < nw; ++i) issue_unit(p, wu0 + i, ring + i * kSlotStride, &full[warp][i]);
   }
   __syncwarp();
+  float sc = 0.f;
+  uint32_t z = 0u;
+  if (active) load_meta(p, wu0, lane, sc, z);  // weights only: no dependency on earlier kernels
   pdl_wait_prior_grids();  // activations, outputs and workspace follow the stream order
 
   const int mcount = min(MT, p.M - p.m0);
   const uint16_t* xrow[MT];
+  if (XS) {  // x' rows of this pass -> shared memory, one bulk copy per row
+    uint16_t* xs = reinterpret_cast<uint16_t*>(ring_smem + ring_bytes(NW));
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(&xbar, (unsigned)(mcount * p.K * 2));
+      for (int m = 0; m < mcount; ++m) bulk_g2s(xs + m * p.K, p.x + (size_t)(p.m0 + m) * p.K, (unsigned)(p.K * 2), &xbar);
+    }
 #pragma unroll
-  for (int m = 0; m < MT; ++m) xrow[m] = p.x + (size_t)(p.m0 + min(m, mcount - 1)) * p.K;
-  float sc = 0.f;
-  uint32_t z = 0u;
-  if (active) load_meta(p, wu0, lane, sc, z);
+    for (int m = 0; m < MT; ++m) xrow[m] = xs + min(m, mcount - 1) * p.K;
+  } else {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) xrow[m] = p.x + (size_t)(p.m0 + min(m, mcount - 1)) * p.K;
+  }
   const int rb_f = active ? wu0 / G : -1;  // the only division of the main path
   const int g0 = active ? wu0 - rb_f * G : 0;
 
   bool ok = true;
+  if (XS && active) ok = __all_sync(0xFFFFFFFFu, mbar_wait_backoff(&xbar, 0u, p.status));
   int rb = rb_f, g = g0, rb_l = rb_f;
   int t = 0;  // units of this warp consumed so far
   while (t < nw && ok) {  // segments: the units of one row block inside this warp's range
@@ -208,7 +229,7 @@ __global__ void __launch_bounds__(kGemvThreads, (MT == 1 ? 4 : MT == 2 ? 2 : 1))
     for (int i = 0; i < seg; ++i, ++t) {
       const int si = t & (kRing - 1);
       uint8_t* slot = ring + si * kSlotStride;
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[warp][si], (unsigned)(t / kRing) & 1u, p.status));
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait_backoff(&full[warp][si], (unsigned)(t / kRing) & 1u, p.status));
       if (!ok) break;  // warp-uniform
       float scn = 0.f;
       uint32_t zn = 0u;
@@ -253,7 +274,7 @@ __global__ void __launch_bounds__(kGemvThreads, (MT == 1 ? 4 : MT == 2 ? 2 : 1))
     float sum[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) sum[m] = 0.f;
-    for (int j = warp; j < kGemvWarps; ++j) {
+    for (int j = warp; j < NW; ++j) {
       const int j0 = cu0 + wq * j + min(j, wr), jn = wq + (j < wr ? 1 : 0);
       if (j0 >= b) break;
       if (jn == 0) continue;
@@ -277,85 +298,25 @@ __global__ void __launch_bounds__(kGemvThreads, (MT == 1 ? 4 : MT == 2 ? 2 : 1))
 #ifndef AWQ_GEMV_WHOLE_RB_MAX_UNITS
 #define AWQ_GEMV_WHOLE_RB_MAX_UNITS 48
 #endif
+#ifndef AWQ_GEMV_BIG_CTA_WARPS  // warps of the one-row-block-per-CTA plan: 16 or 32
+#define AWQ_GEMV_BIG_CTA_WARPS 16
+#endif
+#ifndef AWQ_GEMV_STAGE_X  // stage activations in shared memory when they fit
+#define AWQ_GEMV_STAGE_X 1
+#endif
 
 namespace {
 
 int pick_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
-template <int MT>
-int resident_ctas_mt() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  if (cached[dev] == 0) {
-    int occ = 0;
-    cudaFuncSetAttribute(gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingBytes);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<MT>, kGemvThreads, kRingBytes) !=
-            cudaSuccess || occ < 1)
-      occ = 1;
-    cached[dev] = occ < AWQ_GEMV_CTAS_PER_SM ? occ : AWQ_GEMV_CTAS_PER_SM;
-  }
-  return cached[dev];
-}
-
-// CTAs of one GEMV launch per SM: all resident at once (at most AWQ_GEMV_CTAS_PER_SM).
-int resident_ctas(int MT) {
-  switch (MT) {
-    case 1: return resident_ctas_mt<1>();
-    case 2: return resident_ctas_mt<2>();
-    case 4: return resident_ctas_mt<4>();
-    default: return resident_ctas_mt<8>();
-  }
-}
-
-struct GemvPlan {
-  int MT, RB, G, S, Np, P;
-  int U, q, r;
-  size_t part_bytes;
-};
-
-// P CTAs share the U units.  When the row blocks are short (G small) and numerous enough to occupy at
-// least half the SMs, every CTA takes one whole row block, so no partial sum leaves a CTA; otherwise
-// the units are spread evenly over AWQ_GEMV_CTAS_PER_SM CTAs per SM and the row blocks cut by CTA
-// boundaries are combined in the workspace.
-GemvPlan plan_gemv(int M, int N, int K) {
-  GemvPlan pl{};
-  pl.MT = pick_mt(M);
-  pl.Np = (N + 31) / 32 * 32;
-  pl.RB = pl.Np / 32;
-  pl.G = K / 128;
-  pl.U = pl.RB * pl.G;
-  int p_bal = num_sms() * resident_ctas(pl.MT);
-  const int by_units = pl.U / kGemvWarps > 0 ? pl.U / kGemvWarps : 1;
-  if (p_bal > by_units) p_bal = by_units;
-  if (pl.RB <= p_bal && 2 * pl.RB >= num_sms() && pl.G <= AWQ_GEMV_WHOLE_RB_MAX_UNITS) {
-    pl.P = pl.RB;
-    pl.S = 1;
-    pl.part_bytes = 0;
-  } else {
-    pl.P = p_bal;
-    const int L = pl.U / pl.P;  // >= 1 units per CTA
-    pl.S = pl.G >= 2 ? (pl.G - 2) / L + 2 : 1;
-    pl.part_bytes = (size_t)pl.RB * pl.S * 32 * pl.MT * sizeof(float);
-  }
-  return pl;
-}
-
-}  // namespace
-
-size_t gemv_workspace_bytes(int M, int N, int K) {
-  const GemvPlan pl = plan_gemv(M, N, K);
-  return pl.part_bytes == 0 ? 0 : kWorkspaceCounterBytes + pl.part_bytes;
-}
-
-template <int MT>
+template <int MT, int NW, bool XS>
 bool gemv_smem_attr() {
   static bool done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(gemv_kernel<MT, NW, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ring_bytes(NW) + (XS ? kXsMaxBytes : 0)) != cudaSuccess)
       return false;
     done[dev] = true;
   }
@@ -363,9 +324,109 @@ bool gemv_smem_attr() {
 }
 
 template <int MT>
+int resident_ctas_mt() {  // 8-warp CTAs of one launch resident per SM (at most AWQ_GEMV_CTAS_PER_SM)
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int occ = 0;
+    // sized for the activations staged in shared memory (the larger of the two variants)
+    gemv_smem_attr<MT, 8, true>();
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<MT, 8, true>, 8 * 32,
+                                                      ring_bytes(8) + kXsMaxBytes) != cudaSuccess ||
+        occ < 1)
+      occ = 1;
+    cached[dev] = occ < AWQ_GEMV_CTAS_PER_SM ? occ : AWQ_GEMV_CTAS_PER_SM;
+  }
+  return cached[dev];
+}
+
+int resident_ctas(int MT) {
+  switch (MT) {
+    case 1: return resident_ctas_mt<1>();
+    default: return resident_ctas_mt<2>();
+  }
+}
+int resident_ctas_big(int MT) {  // MT 4 and 8 never stage activations
+  static int cached[64][2] = {{0}};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  const int i = MT == 4 ? 0 : 1;
+  if (cached[dev][i] == 0) {
+    int occ = 0;
+    cudaError_t e;
+    if (MT == 4) {
+      gemv_smem_attr<4, 8, false>();
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<4, 8, false>, 256, ring_bytes(8));
+    } else {
+      gemv_smem_attr<8, 8, false>();
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<8, 8, false>, 256, ring_bytes(8));
+    }
+    if (e != cudaSuccess || occ < 1) occ = 1;
+    cached[dev][i] = occ < AWQ_GEMV_CTAS_PER_SM ? occ : AWQ_GEMV_CTAS_PER_SM;
+  }
+  return cached[dev][i];
+}
+
+struct GemvPlan {
+  int MT, NW, RB, G, S, Np, P;
+  bool xs;  // activations staged in shared memory
+  int U, q, r;
+  size_t part_bytes;
+};
+
+// Three shapes of work, chosen so that all CTAs of a launch are resident at once:
+//  - at most one row block per SM (and M <= 2): one 16-warp CTA per row block; its warps split the
+//    row block's groups and combine in shared memory -- no partial sum leaves a CTA;
+//  - short row blocks (G <= 48) that fit the 8-warp CTAs resident on all SMs: one 8-warp CTA per row
+//    block, likewise self-contained;
+//  - otherwise the units are spread evenly over all resident 8-warp CTAs and the row blocks cut by CTA
+//    boundaries are combined in the workspace.
+GemvPlan plan_gemv(int M, int N, int K) {
+  GemvPlan pl{};
+  pl.MT = pick_mt(M);
+  pl.Np = (N + 31) / 32 * 32;
+  pl.RB = pl.Np / 32;
+  pl.G = K / 128;
+  pl.U = pl.RB * pl.G;
+  const int sms = num_sms();
+  pl.S = 1;
+  pl.part_bytes = 0;
+  if (pl.MT <= 2 && pl.RB <= sms) {
+    pl.NW = AWQ_GEMV_BIG_CTA_WARPS;
+    pl.P = pl.RB;
+  } else {
+    pl.NW = 8;
+    int p_bal = sms * (pl.MT <= 2 ? resident_ctas(pl.MT) : resident_ctas_big(pl.MT));
+    const int by_units = pl.U / 8 > 0 ? pl.U / 8 : 1;
+    if (p_bal > by_units) p_bal = by_units;
+    if (pl.RB <= p_bal && pl.G <= AWQ_GEMV_WHOLE_RB_MAX_UNITS) {
+      pl.P = pl.RB;
+    } else {
+      pl.P = p_bal;
+      const int L = pl.U / pl.P;  // >= 1 units per CTA
+      pl.S = pl.G >= 2 ? (pl.G - 2) / L + 2 : 1;
+      pl.part_bytes = (size_t)pl.RB * pl.S * 32 * pl.MT * sizeof(float);
+    }
+  }
+  pl.q = pl.U / pl.P;
+  pl.r = pl.U % pl.P;
+  pl.xs = AWQ_GEMV_STAGE_X && pl.MT <= 2 && pl.MT * K * 2 <= kXsMaxBytes;
+  return pl;
+}
+
+template <int MT, int NW, bool XS>
 cudaError_t launch_mt(const GemvParams& p, cudaStream_t st) {
-  if (!gemv_smem_attr<MT>()) return cudaErrorInvalidValue;
-  return launch_pdl(gemv_kernel<MT>, dim3((unsigned)p.P), dim3(kGemvThreads), (size_t)kRingBytes, st, p);
+  if (!gemv_smem_attr<MT, NW, XS>()) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)ring_bytes(NW) + (XS ? (size_t)MT * p.K * 2 : 0);
+  return launch_pdl(gemv_kernel<MT, NW, XS>, dim3((unsigned)p.P), dim3(NW * 32), smem, st, p);
+}
+
+}  // namespace
+
+size_t gemv_workspace_bytes(int M, int N, int K) {
+  const GemvPlan pl = plan_gemv(M, N, K);
+  return pl.part_bytes == 0 ? 0 : kWorkspaceCounterBytes + pl.part_bytes;
 }
 
 awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
@@ -383,10 +444,11 @@ awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
   p.y = y;
   p.ws_cnt = static_cast<unsigned*>(ws);
   p.ws_part = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWorkspaceCounterBytes) : nullptr;
+  p.status = dev_status;
   p.U = pl.U;
   p.P = pl.P;
-  p.q = pl.U / pl.P;
-  p.r = pl.U % pl.P;
+  p.q = pl.q;
+  p.r = pl.r;
   p.M = M;
   p.N = N;
   p.Np = pl.Np;
@@ -394,16 +456,22 @@ awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
   p.G = pl.G;
   p.RB = pl.RB;
   p.S = pl.S;
-  p.status = dev_status;
   // passes of MT rows run one after the other on the stream and share the workspace
   for (int m0 = 0; m0 < M; m0 += pl.MT) {
     p.m0 = m0;
     cudaError_t e;
-    switch (pl.MT) {
-      case 1: e = launch_mt<1>(p, st); break;
-      case 2: e = launch_mt<2>(p, st); break;
-      case 4: e = launch_mt<4>(p, st); break;
-      default: e = launch_mt<8>(p, st); break;
+    if (pl.NW == 16 || pl.NW == 32) {
+      constexpr int BW = AWQ_GEMV_BIG_CTA_WARPS;
+      static_assert(ring_bytes(BW) + kXsMaxBytes <= 227 * 1024, "GEMV shared memory over the per-CTA limit");
+      if (pl.MT == 1) e = pl.xs ? launch_mt<1, BW, true>(p, st) : launch_mt<1, BW, false>(p, st);
+      else e = pl.xs ? launch_mt<2, BW, true>(p, st) : launch_mt<2, BW, false>(p, st);
+    } else {
+      switch (pl.MT) {
+        case 1: e = pl.xs ? launch_mt<1, 8, true>(p, st) : launch_mt<1, 8, false>(p, st); break;
+        case 2: e = pl.xs ? launch_mt<2, 8, true>(p, st) : launch_mt<2, 8, false>(p, st); break;
+        case 4: e = launch_mt<4, 8, false>(p, st); break;
+        default: e = launch_mt<8, 8, false>(p, st); break;
+      }
     }
     if (e != cudaSuccess) return AWQ_ERR_CUDA;
   }
