@@ -189,7 +189,9 @@ def summarize_clock_lines(lines):
 class DecodeStack:
     """32 layers x 7 packed linears, inputs x' and outputs y resident in HBM, one CUDA graph per step."""
 
-    def __init__(self, device, seed=0, M=1, layers=LAYERS):
+    def __init__(self, device, seed=0, M=1, layers=LAYERS, inputs_fn=None):
+        """inputs_fn(layer, linear, M, N, K) -> (W, xcal, x) fp16 device tensors; default: the seeded
+        device generator of the synthetic workload."""
         import torch
         import synth
         import weight_only_int4_05_b200 as W4
@@ -203,8 +205,11 @@ class DecodeStack:
         self.y_all = torch.empty(self.d2h_elems, dtype=torch.float16, device=device)
         xo = yo = 0
         for idx, (li, name, K, N) in enumerate(shapes):
-            tid = synth.tensor_id(2, li, DECODE_SHAPES.index((name, K, N)), 0)
-            Wt, xcal, x = synth.device_linear_inputs(seed, tid, M, N, K, device)
+            j = DECODE_SHAPES.index((name, K, N))
+            if inputs_fn is None:
+                Wt, xcal, x = synth.device_linear_inputs(seed, synth.tensor_id(2, li, j, 0), M, N, K, device)
+            else:
+                Wt, xcal, x = inputs_fn(li, j, M, N, K)
             s = W4.awq_act_scale(xcal)
             pw = W4.awq_pack(Wt, s)
             xv = self.x_all[xo:xo + M * K].view(M, K)
@@ -521,6 +526,34 @@ def run_gpu(args):
     return 0
 
 
+def run_profile_case(args):
+    """One linear layer launched `warmup + steps` times eagerly on enough weight copies to exceed L2:
+    the small case for detailed ncu captures.  spec = "gemv:K:N:M" or "gemm:K:N:M"."""
+    import torch
+    import synth
+    import weight_only_int4_05_b200 as W4
+
+    mode, K, N, M = args.profile_case.split(":")
+    K, N, M = int(K), int(N), int(M)
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    W4._lib.load()
+    Wt, xcal, x = synth.device_linear_inputs(0, synth.tensor_id(5, 0, 0, 0), M, N, K, device)
+    s = W4.awq_act_scale(xcal)
+    xp = W4.awq_apply_inv_scale(x, s)
+    copies = max(2, -(-256 * 2**20 // (N * K // 2)))  # > 2 x L2 of packed weights
+    pws = [W4.awq_pack(Wt, s) for _ in range(copies)]
+    del Wt, xcal, x
+    y = torch.empty((M, N), dtype=torch.float16, device=device)
+    fn = {"gemv": W4.w4a16_gemv, "gemm": W4.w4a16_gemm}[mode]
+    for i in range(args.warmup + args.steps):
+        fn(xp, pws[i % copies], out=y)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": args.profile_case, "launches": args.warmup + args.steps,
+                      "copies": copies, "device_status": W4.awq_last_device_status()}))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -528,11 +561,15 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", default=None, metavar="MODE:K:N:M",
+                    help="launch one linear (gemv or gemm) warmup+steps times for an ncu capture, no timing")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_case:
+        return run_profile_case(args)
     return run_gpu(args)
 
 
