@@ -204,6 +204,17 @@ size_t w4a16_workspace_bytes(int mode, int M, int N, int K, int g);
  */
 awq_status awq_last_device_status(awq_stream_t stream);
 
+/*
+ * awq_selftest_wait_timeout -- check of the timeout path above; the pages have no counterpart.
+ * Launches one kernel of one thread that waits on a shared-memory mbarrier phase nothing completes,
+ * with the bounded wait helper of the GEMM (backoff = 0: polling) or of the GEMV (backoff != 0:
+ * polling with nanosleep).  After about 2 s the wait gives up, the device status word is set (so the
+ * next awq_last_device_status returns AWQ_ERR_DEVICE_TIMEOUT) and the kernel writes 1 to *d_returned
+ * (2 would mean the wait completed).  The CUDA context stays usable.  Device memory: d_returned, one
+ * uint32_t, written.  Errors: AWQ_ERR_INVALID_ARG if d_returned is NULL, AWQ_ERR_CUDA on a launch failure.
+ */
+awq_status awq_selftest_wait_timeout(int backoff, uint32_t* d_returned, awq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -98,3 +98,7 @@ def test_pack_and_prep_argument_checks(L):
 def test_workspace_query_rejects_bad_sizes(L):
     assert L.w4a16_workspace_bytes(1, 1, 12, 512, 128) == 2**64 - 1
     assert L.w4a16_workspace_bytes(9, 1, 256, 512, 128) == 2**64 - 1
+
+
+def test_selftest_rejects_null_output(L):
+    assert L.awq_selftest_wait_timeout(0, None, None) == 1  # AWQ_ERR_INVALID_ARG, nothing launched

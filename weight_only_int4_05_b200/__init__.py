@@ -25,6 +25,7 @@ __all__ = [
     "AwqError", "PackedWeight", "GROUP", "awq_packed_sizes", "awq_act_scale", "awq_apply_inv_scale", "awq_pack",
     "w4a16_gemv", "w4a16_gemm", "w4a16_linear", "w4a16_gemv_max_m", "w4a16_workspace_bytes",
     "awq_last_device_status", "reserve_workspace", "lib_path", "w4a16_gemv_noalloc",
+    "awq_selftest_wait_timeout",
 ]
 
 
@@ -166,3 +167,14 @@ def w4a16_gemv_max_m(N: int, K: int) -> int:
 def awq_last_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
     st = torch.cuda.current_stream() if stream is None else stream
     return int(_lib.load().awq_last_device_status(ctypes.c_void_p(st.cuda_stream)))
+
+
+def awq_selftest_wait_timeout(backoff: bool = False) -> int:
+    """Runs the library's bounded-wait timeout check (about 2 s) on the current device.  Returns what the
+    kernel wrote: 1 when the wait gave up and returned, 2 if it completed.  The device status word is
+    left set; awq_last_device_status() then reports AWQ_ERR_DEVICE_TIMEOUT and clears it."""
+    out = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = _lib.load().awq_selftest_wait_timeout(int(bool(backoff)), ctypes.c_void_p(out.data_ptr()),
+                                               _stream(out.device))
+    _lib.check(st, "awq_selftest_wait_timeout")
+    return int(out.item())
