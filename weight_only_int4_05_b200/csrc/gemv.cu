@@ -156,10 +156,16 @@ __device__ __forceinline__ void cross_cta_combine(const GemvParams& p, int r, in
   if (lane == 0) p.ws_cnt[r] = 0u;
 }
 
+#ifndef AWQ_GEMV_MINB_MT1
+#define AWQ_GEMV_MINB_MT1 3
+#endif
+#ifndef AWQ_GEMV_META_AHEAD
+#define AWQ_GEMV_META_AHEAD 2
+#endif
 // NW warps per CTA: 8, 16 or 32.  A 16-warp CTA takes half an SM (64 registers per thread), so the
 // next kernel's CTAs can already be resident beside it; a 32-warp CTA takes a whole SM.
 template <int MT, int NW, bool XS>
-__global__ void __launch_bounds__(NW * 32, (NW == 32 ? 1 : NW == 16 ? 2 : MT == 1 ? 4 : MT == 2 ? 2 : 1))
+__global__ void __launch_bounds__(NW * 32, (NW == 32 ? 1 : NW == 16 ? 2 : MT == 1 ? AWQ_GEMV_MINB_MT1 : MT == 2 ? 2 : 1))
     gemv_kernel(const GemvParams p) {
   extern __shared__ __align__(128) uint8_t ring_smem[];
   __shared__ __align__(8) uint64_t full[NW][kRing];
@@ -194,9 +200,10 @@ __global__ void __launch_bounds__(NW * 32, (NW == 32 ? 1 : NW == 16 ? 2 : MT == 
     for (int i = 0; i < kRing && i < nw; ++i) issue_unit(p, wu0 + i, ring + i * kSlotStride, &full[warp][i]);
   }
   __syncwarp();
-  float sc = 0.f;
-  uint32_t z = 0u;
+  float sc = 0.f, sc1 = 0.f;
+  uint32_t z = 0u, z1 = 0u;
   if (active) load_meta(p, wu0, lane, sc, z);  // weights only: no dependency on earlier kernels
+  if (AWQ_GEMV_META_AHEAD == 2 && nw > 1) load_meta(p, wu0 + 1, lane, sc1, z1);
   pdl_wait_prior_grids();  // activations, outputs and workspace follow the stream order
 
   const int mcount = min(MT, p.M - p.m0);
@@ -233,7 +240,8 @@ __global__ void __launch_bounds__(NW * 32, (NW == 32 ? 1 : NW == 16 ? 2 : MT == 
       if (!ok) break;  // warp-uniform
       float scn = 0.f;
       uint32_t zn = 0u;
-      if (t + 1 < nw) load_meta(p, wu0 + t + 1, lane, scn, zn);  // next unit's scale and zero
+      // scale and zero of a later unit: the next one, or the one after it (two in flight)
+      if (t + AWQ_GEMV_META_AHEAD < nw) load_meta(p, wu0 + t + AWQ_GEMV_META_AHEAD, lane, scn, zn);
       uint4 w[4];
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) w[cc] = *reinterpret_cast<const uint4*>(slot + cc * 512 + lane * 16);
@@ -246,8 +254,15 @@ __global__ void __launch_bounds__(NW * 32, (NW == 32 ? 1 : NW == 16 ? 2 : MT == 
         fence_proxy_async_smem();  // our generic reads of the slot before the async-proxy refill
         issue_unit(p, wu0 + t + kRing, slot, &full[warp][si]);
       }
-      sc = scn;
-      z = zn;
+      if (AWQ_GEMV_META_AHEAD == 2) {
+        sc = sc1;
+        z = z1;
+        sc1 = scn;
+        z1 = zn;
+      } else {
+        sc = scn;
+        z = zn;
+      }
     }
     if (!ok) break;
     if (whole) {
@@ -323,28 +338,39 @@ bool gemv_smem_attr() {
   return true;
 }
 
+#ifndef AWQ_GEMV_OCC_EXACT
+#define AWQ_GEMV_OCC_EXACT 1
+#endif
+// 8-warp CTAs of one launch resident per SM (at most AWQ_GEMV_CTAS_PER_SM), for the shared memory the
+// launch really uses: the rings plus xs_bytes of staged activations (0: not staged).
 template <int MT>
-int resident_ctas_mt() {  // 8-warp CTAs of one launch resident per SM (at most AWQ_GEMV_CTAS_PER_SM)
-  static int cached[64] = {0};
+int resident_ctas_mt(int xs_bytes) {
+  static int cached[64][kXsMaxBytes / 256 + 1] = {{0}};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  if (cached[dev] == 0) {
+  if (!AWQ_GEMV_OCC_EXACT) xs_bytes = kXsMaxBytes;  // sized for the largest staging
+  const int i = (xs_bytes + 255) / 256;
+  if (cached[dev][i] == 0) {
     int occ = 0;
-    // sized for the activations staged in shared memory (the larger of the two variants)
-    gemv_smem_attr<MT, 8, true>();
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<MT, 8, true>, 8 * 32,
-                                                      ring_bytes(8) + kXsMaxBytes) != cudaSuccess ||
-        occ < 1)
-      occ = 1;
-    cached[dev] = occ < AWQ_GEMV_CTAS_PER_SM ? occ : AWQ_GEMV_CTAS_PER_SM;
+    cudaError_t e;
+    if (xs_bytes > 0) {
+      gemv_smem_attr<MT, 8, true>();
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<MT, 8, true>, 8 * 32,
+                                                        ring_bytes(8) + i * 256);
+    } else {
+      gemv_smem_attr<MT, 8, false>();
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<MT, 8, false>, 8 * 32, ring_bytes(8));
+    }
+    if (e != cudaSuccess || occ < 1) occ = 1;
+    cached[dev][i] = occ < AWQ_GEMV_CTAS_PER_SM ? occ : AWQ_GEMV_CTAS_PER_SM;
   }
-  return cached[dev];
+  return cached[dev][i];
 }
 
-int resident_ctas(int MT) {
+int resident_ctas(int MT, int xs_bytes) {
   switch (MT) {
-    case 1: return resident_ctas_mt<1>();
-    default: return resident_ctas_mt<2>();
+    case 1: return resident_ctas_mt<1>(xs_bytes);
+    default: return resident_ctas_mt<2>(xs_bytes);
   }
 }
 int resident_ctas_big(int MT) {  // MT 4 and 8 never stage activations
@@ -397,7 +423,8 @@ GemvPlan plan_gemv(int M, int N, int K) {
     pl.P = pl.RB;
   } else {
     pl.NW = 8;
-    int p_bal = sms * (pl.MT <= 2 ? resident_ctas(pl.MT) : resident_ctas_big(pl.MT));
+    const int xs_bytes = (AWQ_GEMV_STAGE_X && pl.MT <= 2 && pl.MT * K * 2 <= kXsMaxBytes) ? pl.MT * K * 2 : 0;
+    int p_bal = sms * (pl.MT <= 2 ? resident_ctas(pl.MT, xs_bytes) : resident_ctas_big(pl.MT));
     const int by_units = pl.U / 8 > 0 ? pl.U / 8 : 1;
     if (p_bal > by_units) p_bal = by_units;
     if (pl.RB <= p_bal && pl.G <= AWQ_GEMV_WHOLE_RB_MAX_UNITS) {
