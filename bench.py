@@ -554,6 +554,59 @@ def run_profile_case(args):
     return 0
 
 
+CROSSOVER_SHAPES = [(8192, 28672), (28672, 8192)]  # (K, N), 70B-class MLP shapes
+CROSSOVER_MS = [1, 2, 4, 8, 16, 32, 64, 128, 256]
+
+
+def run_crossover(args):
+    """Both modes at every M of the crossover sweep: device time per call (one CUDA graph of calls over
+    weight copies that together exceed L2 several times), and whether w4a16_linear's choice is the faster
+    mode.  Prints one JSON line; no bench metric."""
+    import torch
+    import synth
+    import weight_only_int4_05_b200 as W4
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    W4._lib.load()
+    out = {"crossover": [], "gemv_max_m": None}
+    for i, (K, N) in enumerate(CROSSOVER_SHAPES):
+        Wt, xcal, x = synth.device_linear_inputs(0, synth.tensor_id(4, 0, i, 0), max(CROSSOVER_MS), N, K, device)
+        s = W4.awq_act_scale(xcal)
+        xp_all = W4.awq_apply_inv_scale(x, s)
+        copies = max(2, -(-512 * 2**20 // (N * K // 2)))
+        pws = [W4.awq_pack(Wt, s) for _ in range(copies)]
+        del Wt, xcal, x
+        out["gemv_max_m"] = W4.w4a16_gemv_max_m(N, K)
+        for M in CROSSOVER_MS:
+            xp = xp_all[:M].contiguous()
+            y = torch.empty((M, N), dtype=torch.float16, device=device)
+            need = max(W4.w4a16_workspace_bytes(W4.MODE_GEMV, M, N, K), W4.w4a16_workspace_bytes(W4.MODE_GEMM, M, N, K))
+            ws = W4.reserve_workspace(need, device) if need > 0 else None
+            row = {"K": K, "N": N, "M": M}
+            for mode, fn in (("gemv", W4.w4a16_gemv), ("gemm", W4.w4a16_gemm)):
+                calls = [(lambda p=pw: fn(xp, p, out=y, workspace=ws)) for pw in pws]
+                for c in calls:
+                    c()
+                torch.cuda.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for c in calls:
+                        c()
+                reps = max(3, args.steps)
+                secs, _ = time_steps(g.replay, reps, max(3, args.warmup), device)
+                row[mode + "_us"] = round(secs / reps / len(calls) * 1e6, 2)
+                del g
+            row["faster"] = "gemv" if row["gemv_us"] <= row["gemm_us"] else "gemm"
+            row["chosen"] = "gemv" if M <= out["gemv_max_m"] else "gemm"
+            out["crossover"].append(row)
+        del pws
+        torch.cuda.empty_cache()
+    out["device_status"] = W4.awq_last_device_status()
+    print(json.dumps(out))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -561,6 +614,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--crossover", action="store_true",
+                    help="time both modes at M = 1..256 on the 70B-class shapes (validates the mode choice)")
     ap.add_argument("--profile-case", default=None, metavar="MODE:K:N:M",
                     help="launch one linear (gemv or gemm) warmup+steps times for an ncu capture, no timing")
     args = ap.parse_args(argv)
@@ -570,6 +625,8 @@ def main(argv=None):
         return run_reference(args)
     if args.profile_case:
         return run_profile_case(args)
+    if args.crossover:
+        return run_crossover(args)
     return run_gpu(args)
 
 
