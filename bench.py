@@ -189,9 +189,11 @@ def summarize_clock_lines(lines):
 class DecodeStack:
     """32 layers x 7 packed linears, inputs x' and outputs y resident in HBM, one CUDA graph per step."""
 
-    def __init__(self, device, seed=0, M=1, layers=LAYERS, inputs_fn=None):
+    def __init__(self, device, seed=0, M=1, layers=LAYERS, inputs_fn=None, prefetch=False):
         """inputs_fn(layer, linear, M, N, K) -> (W, xcal, x) fp16 device tensors; default: the seeded
-        device generator of the synthetic workload."""
+        device generator of the synthetic workload.  prefetch: each call passes the next linear's packed
+        weight as an L2 prefetch hint (w4a16_linear_pf)."""
+        self.prefetch = prefetch
         import torch
         import synth
         import weight_only_int4_05_b200 as W4
@@ -232,8 +234,12 @@ class DecodeStack:
         return 1
 
     def eager_step(self):
-        for pw, xv, yv, _, _ in self.entries:
-            self.W4.w4a16_linear(xv, pw, out=yv)
+        n = len(self.entries)
+        for i, (pw, xv, yv, _, _) in enumerate(self.entries):
+            if self.prefetch:  # the next linear of the step (the first one of the next step at the end)
+                self.W4.w4a16_linear_pf(xv, pw, self.entries[(i + 1) % n][0], out=yv)
+            else:
+                self.W4.w4a16_linear(xv, pw, out=yv)
 
     def capture(self):
         torch = self.torch

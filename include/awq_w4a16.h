@@ -186,6 +186,21 @@ awq_status w4a16_linear(const uint16_t* d_x, const uint32_t* d_qweight, const ui
                         const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
                         void* d_workspace, size_t workspace_bytes, awq_stream_t stream);
 
+/*
+ * w4a16_linear_pf -- w4a16_linear with a prefetch hint; the pages have no counterpart (a scheduling
+ * aid for a caller that knows which weight it will use next, e.g. the next linear of a decode step).
+ * In GEMV mode, while the kernel runs, its CTAs also ask for the next_bytes at d_next to be brought
+ * into L2 (cp.async.bulk.prefetch.L2; weights only, issued before the kernel's dependency wait, so
+ * d_next must not be written by earlier work still in flight).  The outputs are exactly those of
+ * w4a16_linear.  In GEMM mode, or with d_next NULL or next_bytes 0, the hint is ignored.
+ *   d_next      device pointer, 16-byte aligned (AWQ_ERR_MISALIGNED otherwise); typically the next
+ *               linear's d_qweight.      next_bytes  a multiple of 16 (AWQ_ERR_INVALID_ARG otherwise).
+ * Other arguments, layout and errors: as w4a16_linear.
+ */
+awq_status w4a16_linear_pf(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                           const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g, void* d_workspace,
+                           size_t workspace_bytes, const void* d_next, size_t next_bytes, awq_stream_t stream);
+
 /* Mode selector used by w4a16_linear: the largest M for which GEMV mode is chosen (4: the crossover
  * measured on B200 for the Llama-3-8B and 70B-class shapes). */
 int w4a16_gemv_max_m(int N, int K);

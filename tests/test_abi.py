@@ -102,3 +102,11 @@ def test_workspace_query_rejects_bad_sizes(L):
 
 def test_selftest_rejects_null_output(L):
     assert L.awq_selftest_wait_timeout(0, None, None) == 1  # AWQ_ERR_INVALID_ARG, nothing launched
+
+
+def test_linear_pf_hint_checks(L):
+    F = ctypes.c_void_p(0x10000)
+    args = (F, F, F, F, F, 1, 256, 512, 128, None, 0)
+    assert L.w4a16_linear_pf(*args, ctypes.c_void_p(0x10008), 64, None) == 3  # misaligned hint
+    assert L.w4a16_linear_pf(*args, F, 24, None) == 1                         # size not a multiple of 16
+    assert L.w4a16_linear_pf(F, F, F, F, F, 0, 256, 512, 128, None, 0, F, 64, None) == 1  # M < 1

@@ -51,7 +51,8 @@ def test_decode_gemv_sweep_full_size(K, N):
     assert_within_tolerance(y.float().cpu().numpy(), y_ref, f"gemv K={K} N={N}")
 
 
-def test_decode_stack_launch_configuration():
+@pytest.mark.parametrize("prefetch", [False, True])
+def test_decode_stack_launch_configuration(prefetch):
     import bench
 
     layers = 2
@@ -62,7 +63,7 @@ def test_decode_stack_launch_configuration():
         cases[(li, j)] = c
         return dev(c.W), dev(c.xcal), dev(c.x)
 
-    stack = bench.DecodeStack(torch.device("cuda", 0), layers=layers, inputs_fn=inputs_fn)
+    stack = bench.DecodeStack(torch.device("cuda", 0), layers=layers, inputs_fn=inputs_fn, prefetch=prefetch)
     stack.capture()
     for _ in range(3):  # replays reuse the workspace; outputs must stay correct
         stack.step()
@@ -96,3 +97,14 @@ def test_crossover_sweep_both_modes(K, N):
         for fn in (W4.w4a16_gemv, W4.w4a16_gemm):
             y = fn(xp, pw).float().cpu().numpy()
             assert_within_tolerance(y[ms, ns], y_ref, f"{fn.__name__} M={M} K={K} N={N}")
+
+
+def test_prefetch_hint_changes_no_output():
+    case = OracleCase(0, 1, 0, 2, 1, 14336, 4096)
+    xp, pw = prep(case)
+    nxt = W4.awq_pack(dev(case.W), None)
+    y0 = W4.w4a16_linear(xp, pw)
+    y1 = W4.w4a16_linear_pf(xp, pw, nxt)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+    assert W4.awq_last_device_status() == 0

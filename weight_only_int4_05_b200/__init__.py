@@ -25,7 +25,7 @@ __all__ = [
     "AwqError", "PackedWeight", "GROUP", "awq_packed_sizes", "awq_act_scale", "awq_apply_inv_scale", "awq_pack",
     "w4a16_gemv", "w4a16_gemm", "w4a16_linear", "w4a16_gemv_max_m", "w4a16_workspace_bytes",
     "awq_last_device_status", "reserve_workspace", "lib_path", "w4a16_gemv_noalloc",
-    "awq_selftest_wait_timeout",
+    "awq_selftest_wait_timeout", "w4a16_linear_pf",
 ]
 
 
@@ -114,7 +114,7 @@ def reserve_workspace(nbytes: int, device=None) -> torch.Tensor:
     return ws
 
 
-def _linear_call(fn_name: str, mode: int, x: torch.Tensor, pw: PackedWeight, out, workspace, g: int):
+def _linear_call(fn_name: str, mode: int, x: torch.Tensor, pw: PackedWeight, out, workspace, g: int, extra=()):
     _need_cuda_fp16(x, "x")
     M, K = x.shape
     if K != pw.K:
@@ -128,7 +128,7 @@ def _linear_call(fn_name: str, mode: int, x: torch.Tensor, pw: PackedWeight, out
     L = _lib.load()
     fn = getattr(L, fn_name)
     st = fn(_p(x), _p(pw.qweight), _p(pw.scales), _p(pw.qzeros), _p(y), M, N, K, g, _p(ws),
-            0 if ws is None else ws.numel() * ws.element_size(), _stream(x.device))
+            0 if ws is None else ws.numel() * ws.element_size(), *extra, _stream(x.device))
     _lib.check(st, fn_name)
     return y
 
@@ -143,6 +143,14 @@ def w4a16_gemm(x, pw: PackedWeight, out=None, workspace=None, g: int = GROUP) ->
 
 def w4a16_linear(x, pw: PackedWeight, out=None, workspace=None, g: int = GROUP) -> torch.Tensor:
     return _linear_call("w4a16_linear", MODE_LINEAR, x, pw, out, workspace, g)
+
+
+def w4a16_linear_pf(x, pw: PackedWeight, next_pw: Optional[PackedWeight], out=None, workspace=None,
+                    g: int = GROUP) -> torch.Tensor:
+    """w4a16_linear that also asks for next_pw's packed codes to be brought into L2 (GEMV mode only)."""
+    nxt = (None, 0) if next_pw is None else (next_pw.qweight, next_pw.qweight.numel() * next_pw.qweight.element_size())
+    extra = (ctypes.c_void_p(0 if nxt[0] is None else nxt[0].data_ptr()), ctypes.c_size_t(nxt[1]))
+    return _linear_call("w4a16_linear_pf", MODE_LINEAR, x, pw, out, workspace, g, extra)
 
 
 def w4a16_gemv_noalloc(x, pw: PackedWeight, out=None, g: int = GROUP) -> torch.Tensor:

@@ -162,6 +162,22 @@ awq_status w4a16_linear(const uint16_t* d_x, const uint32_t* d_qweight, const ui
   return w4a16_gemm(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g, d_workspace, workspace_bytes, stream);
 }
 
+awq_status w4a16_linear_pf(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                           const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g, void* d_workspace,
+                           size_t workspace_bytes, const void* d_next, size_t next_bytes, awq_stream_t stream) {
+  if (d_next == nullptr || next_bytes == 0 || M > w4a16_gemv_max_m(N, K))
+    return w4a16_linear(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g, d_workspace, workspace_bytes, stream);
+  if (!aligned16(d_next)) return AWQ_ERR_MISALIGNED;
+  if (next_bytes % 16 != 0) return AWQ_ERR_INVALID_ARG;
+  awq_status st = check_linear(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g);
+  if (st != AWQ_OK) return st;
+  if (d_workspace && !aligned16(d_workspace)) return AWQ_ERR_MISALIGNED;
+  unsigned* status = device_status_ptr();
+  if (status == nullptr) return AWQ_ERR_CUDA;
+  return gemv_launch(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, d_workspace, workspace_bytes, status,
+                     reinterpret_cast<cudaStream_t>(stream), d_next, next_bytes);
+}
+
 awq_status awq_last_device_status(awq_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return AWQ_ERR_CUDA;

@@ -39,6 +39,9 @@ struct GemvParams {
   float* ws_part;
   unsigned* ws_cnt;
   unsigned* status;  // device status word (bounded waits)
+  const uint8_t* pf;              // optional: bytes to prefetch into L2 for a later call (NULL: none)
+  unsigned long long pf_bytes;    // their size (a multiple of 16)
+  unsigned long long pf_share;    // bytes per CTA (a multiple of 16)
   int U;   // units = RB * G
   int P;   // CTAs sharing the units: CTA c owns q units, plus one more if c < r
   int q, r;
@@ -198,6 +201,13 @@ __global__ void __launch_bounds__(NW * 32, (NW == 32 ? 1 : NW == 16 ? 2 : MT == 
     prefetch_l2_bulk(p.scales + (size_t)wu0 * 32, (unsigned)(nw * 64));
     prefetch_l2_bulk(p.qzeros + (size_t)wu0 * 4, (unsigned)(nw * 16));
     for (int i = 0; i < kRing && i < nw; ++i) issue_unit(p, wu0 + i, ring + i * kSlotStride, &full[warp][i]);
+  }
+  // L2 prefetch of a later call's weights (a caller's hint), spread over the CTAs; weights only.
+  if (p.pf != nullptr && p.m0 == 0 && threadIdx.x == (NW - 1) * 32) {
+    const unsigned long long a = (unsigned long long)c * p.pf_share;
+    const unsigned long long e = a + p.pf_share < p.pf_bytes ? a + p.pf_share : p.pf_bytes;
+    for (unsigned long long o = a; o < e; o += 32768ull)
+      prefetch_l2_bulk(p.pf + o, (unsigned)(e - o < 32768ull ? e - o : 32768ull));
   }
   __syncwarp();
   float sc = 0.f, sc1 = 0.f;
@@ -458,7 +468,7 @@ size_t gemv_workspace_bytes(int M, int N, int K) {
 
 awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
                        uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,
-                       cudaStream_t st) {
+                       cudaStream_t st, const void* pf, size_t pf_bytes) {
   const GemvPlan pl = plan_gemv(M, N, K);
   if ((size_t)pl.RB * 4 > kWorkspaceCounterBytes) return AWQ_ERR_UNSUPPORTED;
   if (pl.part_bytes > 0 && (ws == nullptr || ws_bytes < kWorkspaceCounterBytes + pl.part_bytes))
@@ -472,6 +482,9 @@ awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
   p.ws_cnt = static_cast<unsigned*>(ws);
   p.ws_part = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWorkspaceCounterBytes) : nullptr;
   p.status = dev_status;
+  p.pf = pf_bytes > 0 ? static_cast<const uint8_t*>(pf) : nullptr;
+  p.pf_bytes = pf_bytes;
+  p.pf_share = ((pf_bytes + (size_t)pl.P - 1) / (size_t)pl.P + 15) / 16 * 16;
   p.U = pl.U;
   p.P = pl.P;
   p.q = pl.q;

@@ -45,9 +45,11 @@ awq_status prep_inv_scale_launch(const uint16_t* x, const uint16_t* s, int M, in
 awq_status pack_launch(const uint16_t* W, const uint16_t* s, int N, int K, uint32_t* qw, uint16_t* scales,
                        uint32_t* qz, cudaStream_t st);
 size_t gemv_workspace_bytes(int M, int N, int K);
+// pf / pf_bytes: optional L2 prefetch of another buffer while the GEMV runs (16-byte aligned, size a
+// multiple of 16; NULL / 0 for none).
 awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
                        uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,
-                       cudaStream_t st);
+                       cudaStream_t st, const void* pf = nullptr, size_t pf_bytes = 0);
 unsigned* device_status_ptr();  // address of the device status word on the current device
 size_t gemm_workspace_bytes(int M, int N, int K);
 awq_status gemm_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
