@@ -483,6 +483,16 @@ def run_gpu(args):
     e2e_s, h2d, d2h = e2e_decode(stack, e2e_steps, max(3, args.warmup // 4), device)
     e2e_value = aggregate_value(bytes_step, e2e_steps, world, e2e_s)
 
+    # ---- the same stack with the next linear's weights passed as an L2 prefetch hint
+    stack.prefetch = True
+    stack.capture()
+    pf_s, pf_clocks = time_steps(stack.step, args.steps, args.warmup, device, ClockSampler(gpu_uuid_id(device)))
+    pf_value = aggregate_value(bytes_step, args.steps, world, pf_s)
+    decode_pf = {"value": pf_value, "unit": "GB/s", "ms_per_step": pf_s / args.steps * 1e3,
+                 "frac": pf_value / world / peaks["hbm_gbs"], "steps": args.steps, "clocks": pf_clocks,
+                 "workload": "the same decode stack; every call is w4a16_linear_pf with the next linear's packed "
+                             "codes as the prefetch hint", "gpu_launches": launches * args.steps}
+
     # ---- head 2: prefill GEMM at M=2048
     del stack
     torch.cuda.empty_cache()
@@ -514,7 +524,7 @@ def run_gpu(args):
             "roofline": roofline, "gpu_launches": launches * args.steps, "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
-            "gemm": gemm}
+            "gemm": gemm, "decode_prefetch_hint": decode_pf}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     elif rank == 0:
