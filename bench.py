@@ -37,6 +37,9 @@ if ROOT not in sys.path:
 METRIC = "W4A16 GEMV HBM GB/s (% of peak) at M=1; GEMM TFLOP/s at M=2048"
 DECODE_SHAPES = [("q", 4096, 4096), ("k", 4096, 1024), ("v", 4096, 1024), ("o", 4096, 4096),
                  ("gate", 4096, 14336), ("up", 4096, 14336), ("down", 14336, 4096)]  # (name, K, N)
+# The same layer with the linears that share an input fused into one (the "fused modules" of the
+# AutoAWQ page): q|k|v stacked along N (4096 -> 6144) and gate|up stacked along N (4096 -> 28672).
+FUSED_SHAPES = [("qkv", 4096, 6144), ("o", 4096, 4096), ("gate_up", 4096, 28672), ("down", 14336, 4096)]
 LAYERS = 32
 PREFILL_SHAPES = [(4096, 14336), (14336, 4096), (4096, 4096)]  # (K, N)
 PREFILL_M = 2048
@@ -189,27 +192,29 @@ def summarize_clock_lines(lines):
 class DecodeStack:
     """32 layers x 7 packed linears, inputs x' and outputs y resident in HBM, one CUDA graph per step."""
 
-    def __init__(self, device, seed=0, M=1, layers=LAYERS, inputs_fn=None, prefetch=False):
+    def __init__(self, device, seed=0, M=1, layers=LAYERS, inputs_fn=None, prefetch=False, fused=False):
         """inputs_fn(layer, linear, M, N, K) -> (W, xcal, x) fp16 device tensors; default: the seeded
         device generator of the synthetic workload.  prefetch: each call passes the next linear's packed
-        weight as an L2 prefetch hint (w4a16_linear_pf)."""
+        weight as an L2 prefetch hint (w4a16_linear_pf).  fused: 4 linears per layer (FUSED_SHAPES)."""
         self.prefetch = prefetch
+        layer_shapes = FUSED_SHAPES if fused else DECODE_SHAPES
+        cfg = 6 if fused else 2  # tensor-id namespace of the synthetic inputs
         import torch
         import synth
         import weight_only_int4_05_b200 as W4
 
         self.W4, self.torch, self.device, self.M = W4, torch, device, M
         self.entries = []  # (packed weight, x' view, y view)
-        shapes = [(li, name, K, N) for li in range(layers) for (name, K, N) in DECODE_SHAPES]
+        shapes = [(li, name, K, N) for li in range(layers) for (name, K, N) in layer_shapes]
         self.h2d_elems = sum(M * K for _, _, K, _ in shapes)
         self.d2h_elems = sum(M * N for _, _, _, N in shapes)
         self.x_all = torch.empty(self.h2d_elems, dtype=torch.float16, device=device)
         self.y_all = torch.empty(self.d2h_elems, dtype=torch.float16, device=device)
         xo = yo = 0
         for idx, (li, name, K, N) in enumerate(shapes):
-            j = DECODE_SHAPES.index((name, K, N))
+            j = layer_shapes.index((name, K, N))
             if inputs_fn is None:
-                Wt, xcal, x = synth.device_linear_inputs(seed, synth.tensor_id(2, li, j, 0), M, N, K, device)
+                Wt, xcal, x = synth.device_linear_inputs(seed, synth.tensor_id(cfg, li, j, 0), M, N, K, device)
             else:
                 Wt, xcal, x = inputs_fn(li, j, M, N, K)
             s = W4.awq_act_scale(xcal)
@@ -493,8 +498,22 @@ def run_gpu(args):
                  "workload": "the same decode stack; every call is w4a16_linear_pf with the next linear's packed "
                              "codes as the prefetch hint", "gpu_launches": launches * args.steps}
 
-    # ---- head 2: prefill GEMM at M=2048
+    # ---- the stack with q|k|v and gate|up fused (4 launches per layer, x' read once per fused linear)
     del stack
+    torch.cuda.empty_cache()
+    fstack = DecodeStack(device, fused=True)
+    fstack.capture()
+    f_s, f_clocks = time_steps(fstack.step, args.steps, args.warmup, device, ClockSampler(gpu_uuid_id(device)))
+    f_bytes = fstack.bytes_per_step()
+    f_value = aggregate_value(f_bytes, args.steps, world, f_s)
+    decode_fused = {"value": f_value, "unit": "GB/s", "ms_per_step": f_s / args.steps * 1e3,
+                    "frac": f_value / world / peaks["hbm_gbs"], "steps": args.steps, "clocks": f_clocks,
+                    "bytes_per_step": f_bytes, "gpu_launches": fstack.launches_per_step * args.steps,
+                    "workload": "decode stack with fused linears: 32 layers x {qkv 4096->6144, o 4096->4096, "
+                                "gate_up 4096->28672, down 14336->4096}, M=1, w4a16_linear"}
+    del fstack
+
+    # ---- head 2: prefill GEMM at M=2048
     torch.cuda.empty_cache()
     pre = PrefillGemm(device)
     pre.capture()
@@ -524,7 +543,7 @@ def run_gpu(args):
             "roofline": roofline, "gpu_launches": launches * args.steps, "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
-            "gemm": gemm, "decode_prefetch_hint": decode_pf}
+            "gemm": gemm, "decode_prefetch_hint": decode_pf, "decode_fused": decode_fused}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     elif rank == 0:

@@ -1,8 +1,9 @@
 """GPU parity at the workloads' full sizes, in the launch configurations the benchmark times.
 
   * decode GEMV sweep, M=1, Llama-3-8B shapes: packed arrays bit-exact, every output within tolerance;
-  * decode stack: two layers of the 7-linear stack run as one CUDA graph with programmatic dependent
-    launch and a shared workspace (the benchmark's launch path), every output checked;
+  * decode stack: two layers of the 7-linear stack (also with the prefetch hint) and one layer of the
+    fused 4-linear stack, run as one CUDA graph with programmatic dependent launch and a shared workspace
+    (the benchmark's launch paths), every output checked;
   * prefill GEMM, M=2048: packed arrays bit-exact, sampled outputs (corners + random) within tolerance;
   * crossover sweep, 70B-class shapes: both modes at M = 1 .. 256 on sampled outputs.
 Inputs come from the host generator so that the oracle sees the same values."""
@@ -51,26 +52,28 @@ def test_decode_gemv_sweep_full_size(K, N):
     assert_within_tolerance(y.float().cpu().numpy(), y_ref, f"gemv K={K} N={N}")
 
 
-@pytest.mark.parametrize("prefetch", [False, True])
-def test_decode_stack_launch_configuration(prefetch):
+@pytest.mark.parametrize("prefetch,fused", [(False, False), (True, False), (False, True)])
+def test_decode_stack_launch_configuration(prefetch, fused):
     import bench
 
-    layers = 2
+    layers = 1 if fused else 2
+    shapes = bench.FUSED_SHAPES if fused else bench.DECODE_SHAPES
     cases = {}
 
     def inputs_fn(li, j, M, N, K):
-        c = OracleCase(0, 2, li, j, M, N, K)
+        c = OracleCase(0, 6 if fused else 2, li, j, M, N, K)
         cases[(li, j)] = c
         return dev(c.W), dev(c.xcal), dev(c.x)
 
-    stack = bench.DecodeStack(torch.device("cuda", 0), layers=layers, inputs_fn=inputs_fn, prefetch=prefetch)
+    stack = bench.DecodeStack(torch.device("cuda", 0), layers=layers, inputs_fn=inputs_fn, prefetch=prefetch,
+                              fused=fused)
     stack.capture()
     for _ in range(3):  # replays reuse the workspace; outputs must stay correct
         stack.step()
     torch.cuda.synchronize()
     assert W4.awq_last_device_status() == 0
     for i, (pw, xv, yv, K, N) in enumerate(stack.entries):
-        c = cases[(i // len(bench.DECODE_SHAPES), i % len(bench.DECODE_SHAPES))]
+        c = cases[(i // len(shapes), i % len(shapes))]
         assert np.array_equal(host_u16(xv), c.xp)
         assert_within_tolerance(yv.float().cpu().numpy(), c.y_rows(), f"stack linear {i} K={K} N={N}")
 
