@@ -9,8 +9,8 @@
 //                   fp16 scales and their packed zeros, and a 2-D tensor copy of the x' tile in the 128-byte swizzle
 //                   layout; all complete on full[s].  Weight copies for the first ring are issued before
 //                   griddepcontrol.wait, so they overlap the previous kernel on the stream.
-//   warps 2..       kDequantWG dequant warpgroups take alternate k-blocks, so one warpgroup's latency
-//                   overlaps the other's.  Thread r of a warpgroup owns weight row r of the tile; it turns 64 packed codes into
+//   warps 2..       kDequantWG (4) dequant warpgroups take k-blocks round robin, so one warpgroup's latency
+//                   overlaps the others'.  Thread r of a warpgroup owns weight row r of the tile; it turns 64 packed codes into
 //                   fp16 (q - z) * S (exact q - z by the int4->fp16 bit trick, one rounding for the
 //                   scale) and writes them in the 128-byte swizzle K-major layout the MMA reads, then
 //                   fence.proxy.async + arrive on afull[s].  After the main loop the same warps are
@@ -28,9 +28,9 @@ namespace awq {
 constexpr int kBN = 128;  // weight rows per tile (UMMA M)
 constexpr int kBK = 64;   // channels per k-block (one 128-byte swizzle row of fp16)
 #ifndef AWQ_GEMM_DEQUANT_WG
-#define AWQ_GEMM_DEQUANT_WG 2
+#define AWQ_GEMM_DEQUANT_WG 4
 #endif
-constexpr int kDequantWG = AWQ_GEMM_DEQUANT_WG;            // dequant warpgroups, alternating k-blocks
+constexpr int kDequantWG = AWQ_GEMM_DEQUANT_WG;            // dequant warpgroups, k-blocks round robin
 constexpr int kGemmThreads = 64 + 128 * kDequantWG;
 constexpr int kMaxSmem = 232448;  // opt-in dynamic shared memory per block on sm_100
 
