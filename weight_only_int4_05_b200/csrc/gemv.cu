@@ -13,8 +13,8 @@
 //
 // Streaming.  Each warp owns a contiguous sub-range and streams its codes through its own
 // shared-memory ring of kRing 2 KB unit slots with TMA bulk copies, so the bytes in flight cost no
-// registers; the lanes read each unit's scales and zeros themselves, one unit ahead.  Four 8-warp CTAs
-// per SM keep 32 warps issuing.  Before
+// registers; the lanes read each unit's scales and zeros themselves, two units ahead.  As many 8-warp
+// CTAs per SM as the launch's shared memory allows (3 at K = 4096) keep up to 24 warps issuing.  Before
 // griddepcontrol.wait a kernel touches only its weights -- every warp issues one bulk L2 prefetch of its
 // whole sub-range and fills its ring -- so with programmatic dependent launch the weight stream of the
 // next kernel on the stream starts while this one drains.
