@@ -43,15 +43,21 @@ FUSED_SHAPES = [("qkv", 4096, 6144), ("o", 4096, 4096), ("gate_up", 4096, 28672)
 LAYERS = 32
 PREFILL_SHAPES = [(4096, 14336), (14336, 4096), (4096, 4096)]  # (K, N)
 PREFILL_M = 2048
+CROSSOVER_SHAPES = [(8192, 28672), (28672, 8192)]  # (K, N), 70B-class MLP shapes
+CROSSOVER_MS = [1, 2, 4, 8, 16, 32, 64, 128, 256]
 BYTES_PER_WEIGHT = 0.5 + 2.0 / 128 + 0.5 / 128
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PROFILE_GEMV = os.path.join(ROOT, "profiles", "gemv_kernel_decode_stack.md")
-PROFILE_GEMM = os.path.join(ROOT, "profiles", "gemm_kernel_prefill_m2048.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def gemv_bytes(M, N, K):
     """Algorithmic bytes of one W4A16 linear: packed weight + scales + zeros, x' and y."""
     return N * K * BYTES_PER_WEIGHT + 2 * M * K + 2 * M * N
+
+
+def pack_bytes(N, K):
+    """Algorithmic bytes of one pack: W and s read, packed weight, scales and zeros written."""
+    return 2 * N * K + 2 * K + N * K * BYTES_PER_WEIGHT
 
 
 def decode_step_bytes(M=1):
@@ -76,21 +82,24 @@ def source_hash(files):
     return h.hexdigest()[:16]
 
 
-GEMV_SOURCES = ["weight_only_int4_05_b200/csrc/gemv.cu", "weight_only_int4_05_b200/csrc/common.cuh"]
-GEMM_SOURCES = ["weight_only_int4_05_b200/csrc/gemm.cu", "weight_only_int4_05_b200/csrc/common.cuh"]
+KERNEL_SOURCES = {
+    "gemv_kernel": ["weight_only_int4_05_b200/csrc/gemv.cu", "weight_only_int4_05_b200/csrc/common.cuh"],
+    "gemm_kernel": ["weight_only_int4_05_b200/csrc/gemm.cu", "weight_only_int4_05_b200/csrc/common.cuh"],
+    "pack_kernel": ["weight_only_int4_05_b200/csrc/pack.cu", "weight_only_int4_05_b200/csrc/common.cuh"],
+}
 
 
-def profiled_traffic(profile_path, sources):
-    """DRAM bytes per launch recorded by an ncu capture, or None when the kernel changed since."""
+def profiled_traffic(kernel, path=TRAFFIC_FILE):
+    """DRAM bytes per launch of `kernel` recorded from an ncu capture (profiles/traffic.json), or None when
+    the file lacks it or the kernel's sources changed since the counters were taken."""
     try:
-        text = open(profile_path).read()
-    except OSError:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
         return None
-    m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
-    m_val = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_val or m_hash.group(1) != source_hash(sources):
+    if not rec or rec.get("source_hash") != source_hash(KERNEL_SOURCES[kernel]):
         return None
-    return float(m_val.group(1))
+    return float(rec["bytes_per_launch"])
 
 
 # ------------------------------------------------------------------------------- distributed plumbing
@@ -234,8 +243,8 @@ class DecodeStack:
 
     def _launches(self, K, N):
         W4 = self.W4
-        if self.M <= W4.w4a16_gemv_max_m(N, K):
-            return (self.M + 7) // 8 if self.M > 4 else 1
+        if self.M <= W4.w4a16_gemv_max_m(N, K):  # GEMV passes: one for M <= 8, else passes of 16 rows
+            return 1 if self.M <= 8 else (self.M + 15) // 16
         return 1
 
     def eager_step(self):
@@ -359,34 +368,44 @@ def oracle_sample_linears(seed=0):
 
 
 def oracle_time_linear(d, K, N):
-    """Oracle time (s) of one M=1 linear: every output y[0][n] in fp64 from the quantized weight."""
+    """Oracle seconds of one M=1 linear: (quantize + pack, matmul).  The matmul computes every output
+    y[0][n] in fp64 from the quantized weight."""
     import numpy as np
     from oracle import oracle as O
 
     s = O.act_scale(d["xcal"].view(np.uint16))
     xp = O.inv_scale(d["x"].view(np.uint16), s)
+    t0 = time.perf_counter()
     q, sc, z = O.quantize(d["W"].view(np.uint16), s)
+    O.pack(q, sc, z)
+    t1 = time.perf_counter()
     ms = np.zeros(N, np.int32)
     ns = np.arange(N, dtype=np.int32)
-    t0 = time.perf_counter()
     O.linear_pairs_f64(xp, q, sc, z, ms, ns)
-    return time.perf_counter() - t0
+    return t1 - t0, time.perf_counter() - t1
 
 
 def cpu_baseline(budget_s=12.0):
     """The oracle as it stands, single-threaded on this host, on the first linears of the decode stack
-    until about `budget_s` seconds of oracle time; GB/s of the same algorithmic bytes."""
-    total_t = total_b = 0.0
+    until about `budget_s` seconds of matmul time; GB/s of the same algorithmic bytes.  Quantize + pack is
+    timed separately (setup in the GPU arm as well) and reported beside it."""
+    total_t = total_b = pack_t = pack_b = 0.0
     names = []
     for li, name, K, N, d in oracle_sample_linears():
-        total_t += oracle_time_linear(d, K, N)
+        tp, tm = oracle_time_linear(d, K, N)
+        pack_t += tp
+        pack_b += pack_bytes(N, K)
+        total_t += tm
         total_b += gemv_bytes(1, N, K)
         names.append(f"L{li}.{name}")
         if total_t >= budget_s:
             break
     return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "matmul_s": total_t,
+            "pack": {"value": pack_b / pack_t / 1e9, "unit": "GB/s", "seconds": pack_t},
             "sample": f"{len(names)} linears of the M=1 decode stack ({names[0]}..{names[-1]}), "
-                      f"{total_b / 1e6:.1f} MB of packed weight, {total_t:.1f} s of single-thread oracle time"}
+                      f"{total_b / 1e6:.1f} MB of packed weight: fp64 matmul {total_t:.1f} s and quantize + pack "
+                      f"{pack_t:.1f} s of single-thread oracle time, timed separately"}
 
 
 REF_ROWS_PER_STEP = 256
@@ -451,8 +470,132 @@ def gpu_uuid_id(device):
         return str(device.index)
 
 
+def time_graph_calls(calls, reps, warmup, device):
+    """Device seconds per call of a list of launches captured as one CUDA graph and replayed `reps` times
+    (each replay runs every call once), max over ranks."""
+    import torch
+
+    for c in calls:
+        c()
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c in calls:
+            c()
+    secs, _ = time_steps(g.replay, reps, warmup, device)
+    del g
+    return secs / reps / len(calls)
+
+
+def weight_copies(W4, Wt, s, min_bytes):
+    """Enough packed copies of one weight that together they exceed `min_bytes` (L2 defeated by rotation)."""
+    N, K = Wt.shape
+    per = N * K * BYTES_PER_WEIGHT
+    n = max(2, int(-(-min_bytes // per)))
+    return [W4.awq_pack(Wt, s) for _ in range(n)]
+
+
+def measure_sweep(device, peaks, reps):
+    """Config 1: each M=1 Llama-3-8B linear alone, calls over weight copies totalling 4 x L2, one graph."""
+    import torch
+    import synth
+    import weight_only_int4_05_b200 as W4
+
+    out = []
+    for i, (name, K, N) in enumerate([("q/o", 4096, 4096), ("k/v", 4096, 1024), ("gate/up", 4096, 14336),
+                                      ("down", 14336, 4096)]):
+        Wt, xcal, x = synth.device_linear_inputs(0, synth.tensor_id(1, 0, i, 0), 1, N, K, device)
+        s = W4.awq_act_scale(xcal)
+        xp = W4.awq_apply_inv_scale(x, s)
+        pws = weight_copies(W4, Wt, s, 512 * 2**20)
+        del Wt, xcal, x
+        y = torch.empty((1, N), dtype=torch.float16, device=device)
+        ws = W4.reserve_workspace(max(256, W4.w4a16_workspace_bytes(W4.MODE_GEMV, 1, N, K)), device)
+        calls = [(lambda p=pw: W4.w4a16_linear(xp, p, out=y, workspace=ws)) for pw in pws]
+        sec = time_graph_calls(calls, reps, 3, device)
+        gbs = gemv_bytes(1, N, K) / sec / 1e9
+        out.append({"shape": name, "K": K, "N": N, "M": 1, "us": round(sec * 1e6, 3), "GB/s": round(gbs, 1),
+                    "frac": round(gbs / peaks["hbm_gbs"], 4), "copies": len(pws)})
+        del pws
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure_tiny(device, reps):
+    """Config 0: the tiny layer (M=1, K=512, N=256) -- latency-bound; microseconds per call in a graph."""
+    import torch
+    import synth
+    import weight_only_int4_05_b200 as W4
+
+    Wt, xcal, x = synth.device_linear_inputs(0, synth.tensor_id(0, 0, 0, 0), 1, 256, 512, device)
+    s = W4.awq_act_scale(xcal)
+    xp = W4.awq_apply_inv_scale(x, s)
+    pw = W4.awq_pack(Wt, s)
+    y = torch.empty((1, 256), dtype=torch.float16, device=device)
+    calls = [(lambda: W4.w4a16_linear(xp, pw, out=y))] * 64
+    sec = time_graph_calls(calls, reps, 3, device)
+    return {"shape": "tiny", "K": 512, "N": 256, "M": 1, "us": round(sec * 1e6, 3),
+            "GB/s": round(gemv_bytes(1, 256, 512) / sec / 1e9, 2), "note": "latency-bound; weights stay in L2"}
+
+
+def measure_pack(device, peaks, reps):
+    """awq_pack on the gate/up weight (4096 -> 14336), two different weights alternating (235 MB of fp16
+    input, more than L2); GB/s of W and s read plus the packed arrays written."""
+    import synth
+    import weight_only_int4_05_b200 as W4
+
+    K, N = 4096, 14336
+    inputs = []
+    for i in range(2):
+        Wt, xcal, _ = synth.device_linear_inputs(0, synth.tensor_id(1, 1, 2 + i, 0), 1, N, K, device)
+        inputs.append((Wt, W4.awq_act_scale(xcal)))
+    outs = [W4.awq_pack(*inputs[i]) for i in range(2)]
+    calls = [(lambda i=i: W4.awq_pack(inputs[i][0], inputs[i][1], out=outs[i])) for i in range(2)]
+    sec = time_graph_calls(calls, reps, 3, device)
+    gbs = pack_bytes(N, K) / sec / 1e9
+    return {"value": round(gbs, 1), "unit": "GB/s", "us": round(sec * 1e6, 2), "K": K, "N": N,
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "kernel": "pack_kernel",
+            "bytes_per_launch": pack_bytes(N, K), "traffic": profiled_traffic("pack_kernel"),
+            "workload": "awq_pack of the 4096 -> 14336 weight, two weights alternating (inputs larger than L2)"}
+
+
+def measure_crossover(device, reps):
+    """Config 4: both modes at every M on the two 70B-class shapes; per M the faster mode and the one
+    w4a16_linear picks (calls over weight copies larger than L2, one graph per point)."""
+    import torch
+    import synth
+    import weight_only_int4_05_b200 as W4
+
+    rows = []
+    for i, (K, N) in enumerate(CROSSOVER_SHAPES):
+        Wt, xcal, x = synth.device_linear_inputs(0, synth.tensor_id(4, 0, i, 0), max(CROSSOVER_MS), N, K, device)
+        s = W4.awq_act_scale(xcal)
+        xp_all = W4.awq_apply_inv_scale(x, s)
+        pws = weight_copies(W4, Wt, s, 512 * 2**20)
+        del Wt, xcal, x
+        gmax = W4.w4a16_gemv_max_m(N, K)
+        for M in CROSSOVER_MS:
+            xp = xp_all[:M].contiguous()
+            y = torch.empty((M, N), dtype=torch.float16, device=device)
+            need = max(W4.w4a16_workspace_bytes(W4.MODE_GEMV, M, N, K), W4.w4a16_workspace_bytes(W4.MODE_GEMM, M, N, K))
+            ws = W4.reserve_workspace(max(256, need), device)
+            row = {"K": K, "N": N, "M": M}
+            for mode, fn in (("gemv", W4.w4a16_gemv), ("gemm", W4.w4a16_gemm)):
+                calls = [(lambda p=pw: fn(xp, p, out=y, workspace=ws)) for pw in pws]
+                row[mode + "_us"] = round(time_graph_calls(calls, reps, 2, device) * 1e6, 2)
+            row["faster"] = "gemv" if row["gemv_us"] <= row["gemm_us"] else "gemm"
+            row["chosen"] = "gemv" if M <= gmax else "gemm"
+            row["gemv_GB/s"] = round(gemv_bytes(M, N, K) / row["gemv_us"] / 1e3, 1)
+            row["gemm_TFLOP/s"] = round(2.0 * M * N * K / row["gemm_us"] / 1e6, 1)
+            rows.append(row)
+        del pws
+        torch.cuda.empty_cache()
+    return rows
+
+
 def run_gpu(args):
     import datetime
+    import math
 
     import torch
 
@@ -477,10 +620,9 @@ def run_gpu(args):
     value = aggregate_value(bytes_step, args.steps, world, seconds)
     per_gpu = value / world
     launches = stack.launches_per_step
-    gemv_traffic = profiled_traffic(PROFILE_GEMV, GEMV_SOURCES)
     roofline = {"bound": "hbm", "achieved": per_gpu, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": per_gpu / peaks["hbm_gbs"], "traffic": gemv_traffic,
-                "kernel": "gemv_kernel<1>", "peak_source": peak_src,
+                "frac": per_gpu / peaks["hbm_gbs"], "traffic": profiled_traffic("gemv_kernel"),
+                "kernel": "gemv_kernel<1, true>", "peak_source": peak_src + " (HBM copy, burst)",
                 "bytes_per_launch": bytes_step / launches, "launch_us": seconds / args.steps / launches * 1e6}
 
     # ---- e2e through the public API with host buffers
@@ -512,24 +654,41 @@ def run_gpu(args):
                     "workload": "decode stack with fused linears: 32 layers x {qkv 4096->6144, o 4096->4096, "
                                 "gate_up 4096->28672, down 14336->4096}, M=1, w4a16_linear"}
     del fstack
-
-    # ---- head 2: prefill GEMM at M=2048
     torch.cuda.empty_cache()
+
+    # ---- head 2: prefill GEMM at M=2048, timed over at least 150 ms
     pre = PrefillGemm(device)
     pre.capture()
-    g_steps = max(5, min(100, args.steps // 20))
+    probe_s, _ = time_steps(pre.step, 3, 3, device)
+    g_steps = max(20, math.ceil(0.15 / (probe_s / 3)))
     g_sampler = ClockSampler(gpu_uuid_id(device))
-    g_seconds, g_clocks = time_steps(pre.step, g_steps, max(3, args.warmup // 4), device, g_sampler)
+    g_seconds, g_clocks = time_steps(pre.step, g_steps, 3, device, g_sampler)
     tflops = pre.flops_per_step() * g_steps * world / g_seconds / 1e12
     g_per_gpu = tflops / world
+    per_shape = []
+    for (pw, xp, y, K, N) in pre.entries:
+        sec = time_graph_calls([(lambda pw=pw, xp=xp, y=y: W4.w4a16_gemm(xp, pw, out=y))], max(20, g_steps // 2), 3,
+                               device)
+        per_shape.append({"K": K, "N": N, "M": PREFILL_M, "us": round(sec * 1e6, 2),
+                          "TFLOP/s": round(2.0 * PREFILL_M * N * K / sec / 1e12, 1)})
     gemm = {"value": tflops, "unit": "TFLOP/s", "ms_per_step": g_seconds / g_steps * 1e3, "steps": g_steps,
+            "timed_ms": g_seconds * 1e3,
             "workload": "prefill GEMM M=2048: (K,N) = (4096,14336), (14336,4096), (4096,4096), one step = all three",
-            "gpu_launches": 3 * g_steps, "clocks": g_clocks,
+            "per_shape": per_shape, "gpu_launches": 3 * g_steps, "clocks": g_clocks,
             "roofline": {"bound": "tensor", "achieved": g_per_gpu, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": g_per_gpu / peaks["bf16_tflops"],
                          "frac_of_sustained": g_per_gpu / peaks["bf16_tflops_sustained"],
-                         "traffic": profiled_traffic(PROFILE_GEMM, GEMM_SOURCES), "kernel": "gemm_kernel",
+                         "traffic": profiled_traffic("gemm_kernel"), "kernel": "gemm_kernel",
                          "peak_source": peak_src + " (dense bf16 burst; fp16 runs at the bf16 tensor rate)"}}
+    del pre
+    torch.cuda.empty_cache()
+
+    # ---- the other configurations: the M=1 sweep (config 1), the tiny layer (config 0), pack, crossover
+    reps = max(5, min(50, args.steps // 4))
+    sweep = measure_sweep(device, peaks, reps)
+    tiny = measure_tiny(device, reps)
+    pack = measure_pack(device, peaks, reps)
+    crossover = None if args.no_crossover else measure_crossover(device, max(3, reps // 4))
 
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": seconds / args.steps * 1e3, "higher_is_better": True,
@@ -539,11 +698,13 @@ def run_gpu(args):
                                    "k/v 4096->1024, gate/up 4096->14336, down 14336->4096), M=1, one token per step",
                        "M": 1, "layers": LAYERS, "group_size": 128, "bytes_per_step": bytes_step,
                        "l2": "inputs larger than L2 (3.63 GB of packed weights per step)",
-                       "accumulate": "f32", "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                       "accumulate": "f32 (exact fp16 products on mma.sync, fp32 sums; scale applied in fp32)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": roofline, "gpu_launches": launches * args.steps, "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
-            "gemm": gemm, "decode_prefetch_hint": decode_pf, "decode_fused": decode_fused}
+            "gemm": gemm, "decode_sweep": sweep, "tiny": tiny, "pack": pack, "crossover": crossover,
+            "decode_prefetch_hint": decode_pf, "decode_fused": decode_fused}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     elif rank == 0:
@@ -589,56 +750,19 @@ def run_profile_case(args):
     return 0
 
 
-CROSSOVER_SHAPES = [(8192, 28672), (28672, 8192)]  # (K, N), 70B-class MLP shapes
-CROSSOVER_MS = [1, 2, 4, 8, 16, 32, 64, 128, 256]
 
 
 def run_crossover(args):
-    """Both modes at every M of the crossover sweep: device time per call (one CUDA graph of calls over
-    weight copies that together exceed L2 several times), and whether w4a16_linear's choice is the faster
-    mode.  Prints one JSON line; no bench metric."""
+    """Both modes at every M of the crossover sweep (measure_crossover); prints one JSON line, no bench metric."""
     import torch
-    import synth
     import weight_only_int4_05_b200 as W4
 
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     W4._lib.load()
-    out = {"crossover": [], "gemv_max_m": None}
-    for i, (K, N) in enumerate(CROSSOVER_SHAPES):
-        Wt, xcal, x = synth.device_linear_inputs(0, synth.tensor_id(4, 0, i, 0), max(CROSSOVER_MS), N, K, device)
-        s = W4.awq_act_scale(xcal)
-        xp_all = W4.awq_apply_inv_scale(x, s)
-        copies = max(2, -(-512 * 2**20 // (N * K // 2)))
-        pws = [W4.awq_pack(Wt, s) for _ in range(copies)]
-        del Wt, xcal, x
-        out["gemv_max_m"] = W4.w4a16_gemv_max_m(N, K)
-        for M in CROSSOVER_MS:
-            xp = xp_all[:M].contiguous()
-            y = torch.empty((M, N), dtype=torch.float16, device=device)
-            need = max(W4.w4a16_workspace_bytes(W4.MODE_GEMV, M, N, K), W4.w4a16_workspace_bytes(W4.MODE_GEMM, M, N, K))
-            ws = W4.reserve_workspace(need, device) if need > 0 else None
-            row = {"K": K, "N": N, "M": M}
-            for mode, fn in (("gemv", W4.w4a16_gemv), ("gemm", W4.w4a16_gemm)):
-                calls = [(lambda p=pw: fn(xp, p, out=y, workspace=ws)) for pw in pws]
-                for c in calls:
-                    c()
-                torch.cuda.synchronize()
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    for c in calls:
-                        c()
-                reps = max(3, args.steps)
-                secs, _ = time_steps(g.replay, reps, max(3, args.warmup), device)
-                row[mode + "_us"] = round(secs / reps / len(calls) * 1e6, 2)
-                del g
-            row["faster"] = "gemv" if row["gemv_us"] <= row["gemm_us"] else "gemm"
-            row["chosen"] = "gemv" if M <= out["gemv_max_m"] else "gemm"
-            out["crossover"].append(row)
-        del pws
-        torch.cuda.empty_cache()
-    out["device_status"] = W4.awq_last_device_status()
-    print(json.dumps(out))
+    rows = measure_crossover(device, max(3, args.steps))
+    print(json.dumps({"crossover": rows, "gemv_max_m": W4.w4a16_gemv_max_m(8192, 28672),
+                      "device_status": W4.awq_last_device_status()}))
     return 0
 
 
@@ -649,6 +773,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-crossover", action="store_true", help="leave the crossover sweep out of the bench line")
     ap.add_argument("--crossover", action="store_true",
                     help="time both modes at M = 1..256 on the 70B-class shapes (validates the mode choice)")
     ap.add_argument("--profile-case", default=None, metavar="MODE:K:N:M",
@@ -656,6 +781,11 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus != world:
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch N > 1 ranks with "
+                         f"python -m torch.distributed.run --nproc-per-node N bench.py --gpus N\n")
+        return 2
     if args.impl == "reference":
         return run_reference(args)
     if args.profile_case:

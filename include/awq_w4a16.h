@@ -27,7 +27,12 @@
  *   - NaN or Inf anywhere in W, s, xcal or x is undefined behaviour (not checked).
  *   - Kernels launched by this library call griddepcontrol.wait before they read any activation or
  *     write any output, so they may be launched with programmatic dependent launch; they read only
- *     packed weights before that point.
+ *     packed weights before that point.  Hence the packed weights a linear call reads must not be written
+ *     by work still in flight on the stream, unless that work signals its dependents only when it has
+ *     completed.  awq_pack's kernel never signals early (its dependents start when it has finished), so
+ *     awq_pack followed by a linear call on the same stream, with no synchronisation, is safe.  A caller's
+ *     own kernel that writes packed weights must not trigger programmatic completion before its last write
+ *     to them, or must be separated from the linear call by an event or a host synchronisation.
  *
  * ---------------------------------------------------------------------------------------------------
  * PACKED WEIGHT LAYOUT (this library's own; the producer is awq_pack)
@@ -98,7 +103,8 @@ int awq_version(void);
 
 /*
  * awq_packed_sizes -- byte sizes of the three packed arrays for an N x K weight at group size g
- * (layout above).  Host only; launches nothing.
+ * (layout above; [LLM-AWQ] "quantization flow" fixes w_bit 4 and q_group_size 128, [AWQ/GPTQ] section
+ * 2.3 the saving these sizes realise: 0.51953 B per weight, 74 % below fp16).  Host only; launches nothing.
  * Errors: AWQ_ERR_INVALID_ARG if N < 1, K < 1, K % g != 0 or an output pointer is NULL;
  *         AWQ_ERR_UNSUPPORTED if g != 128.
  */
@@ -154,10 +160,12 @@ awq_status awq_pack(const uint16_t* d_W, const uint16_t* d_s, int N, int K, int 
  * Errors: AWQ_ERR_INVALID_ARG, AWQ_ERR_UNSUPPORTED, AWQ_ERR_MISALIGNED, AWQ_ERR_WORKSPACE, AWQ_ERR_CUDA.
  */
 
-/* w4a16_gemv -- decode path ([AutoAWQ] "GEMV mode", single batch): CUDA-core kernel that streams the
- * packed weights once per 8 rows of x with 128-bit loads, dequantizes in registers and accumulates
- * in fp32; the input channels are split across warps and the partial sums are combined in the
- * workspace.  Any M is accepted (M > 8 runs ceil(M/8) passes). */
+/* w4a16_gemv -- decode path ([AutoAWQ] "GEMV mode", single batch): streams the packed weights once per
+ * pass of up to 16 rows of x' (M <= 8: one pass of 8; larger M: passes of 16) through per-warp shared-memory
+ * rings filled by TMA bulk copies, turns each code into the exact fp16 integer q - z in registers and
+ * contracts it with x' on the tensor cores (mma.sync m16n8k16, exact products, fp32 accumulation); each
+ * group's fp32 sum is multiplied by its scale in fp32.  Units of the weight are spread over the SMs; a row
+ * block split between CTAs is combined in the workspace in a fixed order (results are deterministic). */
 awq_status w4a16_gemv(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
                       const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
                       void* d_workspace, size_t workspace_bytes, awq_stream_t stream);
@@ -181,7 +189,8 @@ awq_status w4a16_gemv_noalloc(const uint16_t* d_x, const uint32_t* d_qweight, co
                               const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
                               awq_stream_t stream);
 
-/* w4a16_linear -- picks GEMV when M <= w4a16_gemv_max_m(N, K), GEMM otherwise, and calls it. */
+/* w4a16_linear -- the mode choice of [AutoAWQ] "quantization parameters" (GEMV mode for a single batch,
+ * GEMM mode for long contexts): picks GEMV when M <= w4a16_gemv_max_m(N, K), GEMM otherwise, and calls it. */
 awq_status w4a16_linear(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
                         const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
                         void* d_workspace, size_t workspace_bytes, awq_stream_t stream);
@@ -201,8 +210,8 @@ awq_status w4a16_linear_pf(const uint16_t* d_x, const uint32_t* d_qweight, const
                            const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g, void* d_workspace,
                            size_t workspace_bytes, const void* d_next, size_t next_bytes, awq_stream_t stream);
 
-/* Mode selector used by w4a16_linear: the largest M for which GEMV mode is chosen (4: the crossover
- * measured on B200 for the Llama-3-8B and 70B-class shapes). */
+/* Mode selector used by w4a16_linear: the largest M for which GEMV mode is chosen (32: the crossover
+ * measured on B200 for the 70B-class shapes). */
 int w4a16_gemv_max_m(int N, int K);
 
 /* Modes for w4a16_workspace_bytes. */

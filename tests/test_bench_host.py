@@ -30,12 +30,25 @@ def test_aggregate_value_counts_every_rank():
 
 
 def test_profiled_traffic_requires_matching_source(tmp_path):
-    p = tmp_path / "prof.md"
-    p.write_text(f"source_hash: {bench.source_hash(bench.GEMV_SOURCES)}\ntraffic_bytes_per_launch: 123.5\n")
-    assert bench.profiled_traffic(str(p), bench.GEMV_SOURCES) == 123.5
-    p.write_text("source_hash: 0000\ntraffic_bytes_per_launch: 123.5\n")
-    assert bench.profiled_traffic(str(p), bench.GEMV_SOURCES) is None
-    assert bench.profiled_traffic(str(tmp_path / "missing.md"), bench.GEMV_SOURCES) is None
+    p = tmp_path / "traffic.json"
+    h = bench.source_hash(bench.KERNEL_SOURCES["gemv_kernel"])
+    p.write_text(json.dumps({"gemv_kernel": {"source_hash": h, "bytes_per_launch": 123.5}}))
+    assert bench.profiled_traffic("gemv_kernel", str(p)) == 123.5
+    assert bench.profiled_traffic("gemm_kernel", str(p)) is None
+    p.write_text(json.dumps({"gemv_kernel": {"source_hash": "0000", "bytes_per_launch": 123.5}}))
+    assert bench.profiled_traffic("gemv_kernel", str(p)) is None
+    assert bench.profiled_traffic("gemv_kernel", str(tmp_path / "missing.json")) is None
+
+
+def test_gpus_flag_must_match_world_size(monkeypatch, capsys):
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    assert bench.main(["--gpus", "8", "--impl", "reference", "--steps", "1"]) == 2
+    assert "WORLD_SIZE" in capsys.readouterr().err
+
+
+def test_pack_and_linear_byte_counts():
+    assert bench.gemv_bytes(1, 14336, 4096) == pytest.approx(14336 * 4096 * 0.51953125 + 2 * 4096 + 2 * 14336)
+    assert bench.pack_bytes(14336, 4096) == pytest.approx(2 * 14336 * 4096 + 2 * 4096 + 14336 * 4096 * 0.51953125)
 
 
 def _free_port():
@@ -79,5 +92,5 @@ def test_reference_arm_silent_on_nonzero_rank(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "2")
     buf = io.StringIO()
     with redirect_stdout(buf):
-        rc = bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+        rc = bench.main(["--gpus", "2", "--impl", "reference", "--steps", "1", "--warmup", "3"])
     assert rc == 0 and buf.getvalue() == ""

@@ -54,6 +54,16 @@ def _need_cuda_fp16(t: torch.Tensor, name: str) -> None:
         raise ValueError(f"{name} must be a contiguous CUDA float16 tensor")
 
 
+def _check_out(out: torch.Tensor, shape, device, name: str = "out") -> None:
+    """A caller-supplied output must be exactly what the kernel writes: a wrong size would become an
+    out-of-bounds device write instead of an error."""
+    _need_cuda_fp16(out, name)
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(out.shape)}, expected {tuple(shape)}")
+    if out.device != torch.device(device):
+        raise ValueError(f"{name} is on {out.device}, expected {device}")
+
+
 def awq_packed_sizes(N: int, K: int, g: int = GROUP):
     L = _lib.load()
     a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
@@ -64,6 +74,8 @@ def awq_packed_sizes(N: int, K: int, g: int = GROUP):
 def awq_act_scale(xcal: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     _need_cuda_fp16(xcal, "xcal")
     R, K = xcal.shape
+    if out is not None:
+        _check_out(out, (K,), xcal.device)
     s = torch.empty(K, dtype=torch.float16, device=xcal.device) if out is None else out
     L = _lib.load()
     _lib.check(L.awq_act_scale(_p(xcal), R, K, _p(s), _stream(xcal.device)), "awq_act_scale")
@@ -74,22 +86,36 @@ def awq_apply_inv_scale(x: torch.Tensor, s: torch.Tensor, out: Optional[torch.Te
     _need_cuda_fp16(x, "x")
     _need_cuda_fp16(s, "s")
     M, K = x.shape
+    if s.shape != (K,):
+        raise ValueError(f"s has shape {tuple(s.shape)}, expected ({K},)")
+    if out is not None:
+        _check_out(out, (M, K), x.device)
     xp = torch.empty_like(x) if out is None else out
     L = _lib.load()
     _lib.check(L.awq_apply_inv_scale(_p(x), _p(s), M, K, _p(xp), _stream(x.device)), "awq_apply_inv_scale")
     return xp
 
 
-def awq_pack(W: torch.Tensor, s: Optional[torch.Tensor] = None, g: int = GROUP) -> PackedWeight:
+def awq_pack(W: torch.Tensor, s: Optional[torch.Tensor] = None, g: int = GROUP,
+             out: Optional[PackedWeight] = None) -> PackedWeight:
+    """Packs W (with s folded in); `out` reuses the three buffers of an earlier PackedWeight of the same shape."""
     _need_cuda_fp16(W, "W")
+    N, K = W.shape
     if s is not None:
         _need_cuda_fp16(s, "s")
-    N, K = W.shape
+        if s.shape != (K,):
+            raise ValueError(f"s has shape {tuple(s.shape)}, expected ({K},)")
     qb, sb, zb = awq_packed_sizes(N, K, g)
     dev = W.device
-    qw = torch.empty(qb // 4, dtype=torch.int32, device=dev)
-    sc = torch.empty(sb // 2, dtype=torch.float16, device=dev)
-    qz = torch.empty(zb // 4, dtype=torch.int32, device=dev)
+    if out is not None:
+        if (out.N, out.K) != (N, K) or out.qweight.numel() * 4 != qb or out.scales.numel() * 2 != sb \
+                or out.qzeros.numel() * 4 != zb or any(t.device != dev for t in out[:3]):
+            raise ValueError("out does not match the packed sizes of W")
+        qw, sc, qz = out.qweight, out.scales, out.qzeros
+    else:
+        qw = torch.empty(qb // 4, dtype=torch.int32, device=dev)
+        sc = torch.empty(sb // 2, dtype=torch.float16, device=dev)
+        qz = torch.empty(zb // 4, dtype=torch.int32, device=dev)
     L = _lib.load()
     _lib.check(L.awq_pack(_p(W), _p(s), N, K, g, _p(qw), _p(sc), _p(qz), _stream(dev)), "awq_pack")
     return PackedWeight(qw, sc, qz, N, K)
@@ -120,6 +146,8 @@ def _linear_call(fn_name: str, mode: int, x: torch.Tensor, pw: PackedWeight, out
     if K != pw.K:
         raise ValueError(f"x has K={K}, weight has K={pw.K}")
     N = pw.N
+    if out is not None:
+        _check_out(out, (M, N), x.device)
     y = torch.empty((M, N), dtype=torch.float16, device=x.device) if out is None else out
     need = w4a16_workspace_bytes(mode, M, N, K, g)
     if need == 2**64 - 1:
@@ -160,6 +188,8 @@ def w4a16_gemv_noalloc(x, pw: PackedWeight, out=None, g: int = GROUP) -> torch.T
     M, K = x.shape
     if K != pw.K:
         raise ValueError(f"x has K={K}, weight has K={pw.K}")
+    if out is not None:
+        _check_out(out, (M, pw.N), x.device)
     y = torch.empty((M, pw.N), dtype=torch.float16, device=x.device) if out is None else out
     L = _lib.load()
     st = L.w4a16_gemv_noalloc(_p(x), _p(pw.qweight), _p(pw.scales), _p(pw.qzeros), _p(y), M, pw.N, K, g,

@@ -39,7 +39,7 @@ unsigned* device_status_ptr() {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-constexpr int kMaxN = 1 << 21;   // packed row blocks index grid.y of the pack kernel
+constexpr int kMaxN = 1 << 21;   // sanity bounds on the sizes (a split linear further needs N / 32 <= 16384)
 constexpr int kMaxK = 1 << 20;
 
 awq_status check_linear(const uint16_t* x, const uint32_t* qw, const uint16_t* sc, const uint32_t* qz,
@@ -146,12 +146,13 @@ awq_status w4a16_gemm(const uint16_t* d_x, const uint32_t* d_qweight, const uint
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
-// Crossover measured on B200 over the Llama-3-8B and 70B-class shapes (M = 1..16): the CUDA-core GEMV
-// is faster up to M = 4 on every shape; from M = 8 the split-K tensor-core GEMM is faster.
+// Crossover measured on B200 over the 70B-class shapes (M = 1 .. 256): the weight-streaming GEMV costs
+// almost the same from M = 1 to 8 (one pass), 1.35x at M = 16 (two 8-row tiles per pass) and 2.7x at M = 32
+// (two passes), and is faster than the tcgen05 GEMM through M = 32; from M = 64 the GEMM is faster.
 int w4a16_gemv_max_m(int N, int K) {
   (void)N;
   (void)K;
-  return 4;
+  return 32;
 }
 
 awq_status w4a16_linear(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,

@@ -65,6 +65,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of the phase with the given parity (for polling several barriers in turn).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Waits for the phase with the given parity to complete.  Gives up after kWaitLimitNs, records a
 // timeout in *status and returns false; the caller then abandons its work and exits cleanly.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsigned* status) {
@@ -200,6 +212,41 @@ __device__ __forceinline__ void named_barrier_sync(unsigned id, unsigned threads
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// ---------------------------------------------------------------- warp-level MMA (register fragments)
+// D = A . B + C for one 16 x 8 x 16 tile: A 16 x 16 fp16 (row major), B 16 x 8 fp16 (column major), C/D fp32.
+// Thread (g = lane / 4, t = lane % 4) holds A rows g and g + 8 at columns {2t, 2t+1} (a0: row g, a1: row
+// g + 8) and {2t+8, 2t+9} (a2: row g, a3: row g + 8); B column g at rows {2t, 2t+1} (b0) and {2t+8, 2t+9}
+// (b1); C/D rows g (c[0], c[1]) and g + 8 (c[2], c[3]) at columns 2t and 2t + 1.  Products are exact in
+// fp32 and accumulate in fp32.
+__device__ __forceinline__ void mma_16816_f32(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------- shared-memory loads by 32-bit address
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint16_t ld_shared_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+// Arrive (count 1) on an mbarrier given by its 32-bit shared address.
+__device__ __forceinline__ void mbar_arrive_addr(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 // ---------------------------------------------------------------- loads
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {  // read-once data: skip L1
   uint4 v;
@@ -247,6 +294,16 @@ __device__ __forceinline__ void word_minus_zero(uint32_t w, __half2 z1024, __hal
   d[2] = __hsub2(u32_as_h2(and_or<0x000F000Fu>(t, magic)), z1024);
   d[3] = __hfma2(u32_as_h2(and_or<0x00F000F0u>(t, magic)), sixteenth, nz64);
 }
+// fp16 64 in both halves: with the nibble in mantissa bits 4..7 ((w & 0x00F000F0) | 0x54005400) each
+// half is exactly 64 + code, since one unit in the last place of 64 is 1/16.
+__device__ __forceinline__ uint32_t magic_64x2() {
+  uint32_t m;
+  asm volatile("mov.b32 %0, 0x54005400;" : "=r"(m));
+  return m;
+}
+// fp16 (64 + z) in both halves, from a zero point 0..15.
+__device__ __forceinline__ __half2 zero_64(uint32_t z) { return u32_as_h2((0x5400u | (z << 4)) * 0x00010001u); }
+
 // fp16 (1024 + z) and -(64 + z), splatted into both halves, from a zero point 0..15.
 __device__ __forceinline__ __half2 zero_1024(uint32_t z) { return u32_as_h2((0x6400u | z) * 0x00010001u); }
 __device__ __forceinline__ __half2 neg_zero_64(uint32_t z) {

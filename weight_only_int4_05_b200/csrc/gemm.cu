@@ -176,7 +176,8 @@ __device__ __forceinline__ void gemm_dequant_epilogue(const GemmParams& p, uint8
   // Every epilogue thread reaches this barrier (its wait is bounded); after it the abort flag is final
   // (the producer and MMA roles are done), so all epilogue warps take the same decision.
   named_barrier_sync(1, 128 * kDequantWG);
-  if (*abort_flag) return;
+  const bool aborted = *abort_flag != 0;
+  if (aborted && p.splits == 1) return;
   const int q = warp & 3;
   const int row = 32 * q + lane;
   const int n = n0 + row;
@@ -200,12 +201,14 @@ __device__ __forceinline__ void gemm_dequant_epilogue(const GemmParams& p, uint8
   const int tile = blockIdx.y * gridDim.x + blockIdx.x;
   float* tile_ws = p.ws_part + (size_t)tile * p.splits * p.BT * 128;
   float* mine = tile_ws + (size_t)blockIdx.z * p.BT * 128;  // [column][row]
-  for (int c0 = 16 * wg; c0 < p.BT; c0 += 16 * kDequantWG) {
-    uint32_t v[16];
-    tmem_ld_32x32b_x16(tq + (uint32_t)c0, v);
-    tmem_wait_ld();
+  if (!aborted) {  // an aborted CTA has no valid accumulator, but still arrives on the tile counter below
+    for (int c0 = 16 * wg; c0 < p.BT; c0 += 16 * kDequantWG) {
+      uint32_t v[16];
+      tmem_ld_32x32b_x16(tq + (uint32_t)c0, v);
+      tmem_wait_ld();
 #pragma unroll
-    for (int i = 0; i < 16; ++i) mine[(size_t)(c0 + i) * 128 + row] = __uint_as_float(v[i]);
+      for (int i = 0; i < 16; ++i) mine[(size_t)(c0 + i) * 128 + row] = __uint_as_float(v[i]);
+    }
   }
   __threadfence();
   named_barrier_sync(1, 128 * kDequantWG);
@@ -213,6 +216,12 @@ __device__ __forceinline__ void gemm_dequant_epilogue(const GemmParams& p, uint8
   if (threadIdx.x == 64) *s_last = atomicAdd(&p.ws_cnt[tile], 1u) == (unsigned)(p.splits - 1);
   named_barrier_sync(1, 128 * kDequantWG);
   if (!*s_last) return;
+  // Every split of the tile has arrived: the counter goes back to zero for the next call whatever
+  // happened (after a timeout the output is invalid and the status word says so).
+  if (aborted) {
+    if (threadIdx.x == 64) p.ws_cnt[tile] = 0u;
+    return;
+  }
   __threadfence();
   for (int c0 = 16 * wg; c0 < p.BT; c0 += 16 * kDequantWG) {
     float acc[16];

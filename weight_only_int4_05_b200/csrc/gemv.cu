@@ -1,51 +1,103 @@
 // gemv.cu -- W4A16 decode kernel ("GEMV mode" of the AutoAWQ page: single batch, top speed).
 //
-// y[m][n] = sum_g S[n][g] * sum_{k in g} (q[n][k] - z[n][g]) * x'[m][k]   for up to MT rows of x' per pass.
+// y[m][n] = sum_g S[n][g] * sum_{k in g} (q[n][k] - z[n][g]) * x'[m][k]   for up to 8 * NT rows of x' per pass.
 //
-// Units.  The packed layout stores each (32-row block rb, 128-channel group g) as 2048 contiguous
-// bytes, so unit u = rb * G + g is one 2 KB stretch and the weight is U = RB * G consecutive units.
-// Each of the P CTAs owns a balanced contiguous range (q = U / P units, one more for the first U % P
-// CTAs); its NW warps split that range into NW balanced contiguous sub-ranges.  Inside a warp, lane r owns row 32*rb + r: a unit is four
-// coalesced 128-bit loads per lane (512 contiguous bytes per warp-instruction), dequantized in registers
-// with the int4->fp16 bit trick, multiplied with x' in packed half2 FMAs (two independent accumulators,
-// 16 products each, flushed to fp32 every 64 channels), scaled by the group's fp16 scale and
-// accumulated in fp32.  No cross-lane reduction is needed: the layout gives each lane a whole row.
+// Units.  The packed layout stores each (32-row block rb, 128-channel group g) as 2048 contiguous bytes of
+// codes, and its 32 scales (64 B) and 32 zero nibbles (16 B) contiguously in the unit-major scale and zero
+// arrays, so unit u = rb * G + g is one stretch of each.  Each of the P CTAs owns a balanced contiguous range
+// of units (q = U / P, one more for the first U % P CTAs); its kNW consumer warps split that range into
+// contiguous sub-ranges, and each consumer warp has its own ring of kRing shared-memory slots.
 //
-// Streaming.  Each warp owns a contiguous sub-range and streams its codes through its own
-// shared-memory ring of kRing 2 KB unit slots with TMA bulk copies, so the bytes in flight cost no
-// registers; the lanes read each unit's scales and zeros themselves, two units ahead.  As many 8-warp
-// CTAs per SM as the launch's shared memory allows (3 at K = 4096) keep up to 24 warps issuing.  Before
-// griddepcontrol.wait a kernel touches only its weights -- every warp issues one bulk L2 prefetch of its
-// whole sub-range and fills its ring -- so with programmatic dependent launch the weight stream of the
-// next kernel on the stream starts while this one drains.
+// Warp roles.  One producer warp per CTA fills every slot with TMA bulk copies -- the codes, scales and zeros
+// of kSU consecutive units, three copies completing on the slot's "full" mbarrier -- and refills a slot when
+// its consumer has released it on the slot's "empty" mbarrier.  Slot j of the CTA (warp j / kRing, ring index j % kRing) is
+// served by producer lane j % 32: a thread completes about one bulk copy per ~770 cycles whatever its size,
+// and a copy waiting behind another one stalls its thread, so spreading the slots over the lanes keeps the
+// copies in parallel and keeps every issue stall off the consumer warps.
 //
-// Combining split row blocks.  A row block wholly inside one warp's sub-range is written directly.  A
-// row block split between warps of one CTA is summed in shared memory, in warp order.  A row block
-// split between CTAs gets one fp32 partial per CTA in the workspace slot (rb, c - first_cta(rb)); the
-// CTA that brings the row block's counter to its final value sums the slots in slot order
-// (deterministic), writes fp16 y and resets the counter to 0 for the next call.
+// Arithmetic: the tensor cores, fp32 accumulation.  One unit is two 16-row halves x 8 steps of
+// mma.sync m16n8k16 (A = weights, 16 rows x 16 channels; B = x', 16 channels x 8 rows of x'; C = fp32).
+// Lane (g = lane / 4, t = lane % 4) reads word t of rows g and g + 8 of each 32-channel chunk c (conflict-
+// free 4-byte shared loads).  The nibble order of a word makes (w & 0x000F000F) | 0x64006400 the fp16 pair
+// (1024 + q) for channels (8t, 8t+1) and (w & 0x00F000F0) | 0x54005400 the pair (64 + q) for (8t+2, 8t+3);
+// the word shifted right by 8 gives channels 8t+4 .. 8t+7 the same way.  One fp16 subtraction of
+// (1024 + z) or (64 + z) turns each pair into the exact integers q - z.  Those four pairs are the thread's
+// A fragment for one MMA: its k slots {2t, 2t+1} and {2t+8, 2t+9} stand for channels 32c + 8t + {0, 1}
+// and + {2, 3} (or + {4..7}), and the B fragment holds x' at the same channels, so every product
+// (q - z) * x' is formed exactly in fp32 and summed in fp32.  Each half runs two independent MMA chains
+// (even and odd chunks).  After the 8 steps of a group the fp32 sum of each row is multiplied by the row's
+// scale and added to the row's fp32 output accumulator.  Nothing is summed in fp16.
+//
+// Before griddepcontrol.wait a kernel touches only its weights: the producer fills the first kRing slots of
+// every consumer before the wait, so with programmatic dependent launch the next kernel's weight stream
+// starts while the previous kernel still runs.  After the wait, x' (the rows of this pass) is staged in
+// shared memory by one TMA copy per row when it fits, with a row pitch padded so that rows fall in different
+// banks; otherwise each lane reads its B fragments (64 bytes per unit) from global memory one unit ahead.
+//
+// Combining split row blocks.  A row block wholly inside one warp's sub-range is written directly.  A row
+// block split between warps of one CTA is summed in shared memory, in warp order.  A row block split between
+// CTAs gets one fp32 partial per CTA in the workspace slot (rb, c - first_cta(rb)); the CTA that brings the
+// row block's counter to its final value sums the slots in slot order (deterministic), writes fp16 y and
+// resets the counter to 0 for the next call.  A CTA whose bounded wait ran out still takes part in this
+// protocol (with invalid values), so the counters are zero again after every call.
 #include "common.cuh"
 #include "internal.h"
 
 namespace awq {
 
+// ------------------------------------------------------------------------------------------ constants
+constexpr int kUnitCodeBytes = 2048;
+#ifndef AWQ_GEMV_SLOT_UNITS
+#define AWQ_GEMV_SLOT_UNITS 4
+#endif
+// A ring slot holds kSU consecutive units of a warp's range: their codes (kSU x 2 KB), then their scales
+// (kSU x 64 B), then their zeros (kSU x 16 B) -- three copies per slot, since consecutive units are
+// contiguous in all three arrays.  Few large copies keep the bytes in flight high: a thread gets only about
+// one bulk copy serviced at a time, and under load a copy takes the full memory latency.
+constexpr int kSU = AWQ_GEMV_SLOT_UNITS;
+static_assert((kSU & (kSU - 1)) == 0 && kSU >= 1 && kSU <= 8, "units per slot: 1, 2, 4 or 8");
+constexpr int kSlotScaleOff = kSU * kUnitCodeBytes;
+constexpr int kSlotZeroOff = kSlotScaleOff + kSU * 64;
+constexpr int kSlotStride = (kSU * 2128 + 127) / 128 * 128;
+#ifndef AWQ_GEMV_RING
+#define AWQ_GEMV_RING 2
+#endif
+constexpr int kRing = AWQ_GEMV_RING;  // slots per consumer warp (power of two)
+static_assert((kRing & (kRing - 1)) == 0, "ring depth must be a power of two");
+#ifndef AWQ_GEMV_WARPS
+#define AWQ_GEMV_WARPS 8
+#endif
+constexpr int kNW = AWQ_GEMV_WARPS;  // consumer warps per CTA (power of two); one producer warp besides
+#ifndef AWQ_GEMV_L2_PREFETCH  // bulk L2 prefetch of each warp's range before the wait (measured slower: off)
+#define AWQ_GEMV_L2_PREFETCH 0
+#endif
+static_assert((kNW & (kNW - 1)) == 0 && kNW >= 2 && kNW <= 16, "consumer warps per CTA: 2, 4, 8 or 16");
+constexpr int kSlots = kNW * kRing;
+constexpr int kThreads = (kNW + 1) * 32;
+constexpr int kRingBytes = kSlots * kSlotStride;
+static_assert(kRingBytes <= 160 * 1024, "rings too large for shared memory");
+constexpr int kXsMaxBytes = 36 * 1024;  // x' of one pass staged in shared memory when it fits
+constexpr int kXPad = 32;                // halves of padding per staged row: rows 64 B apart fall in other banks
+constexpr int kMaxDynSmem = 232448 - 2048;  // opt-in shared memory per block, less the static barriers
 
 struct GemvParams {
   const uint16_t* x;
-  const uint4* qw;
-  const __half* scales;
+  const uint8_t* qw;
+  const uint16_t* scales;
   const uint32_t* qzeros;
   uint16_t* y;
   float* ws_part;
   unsigned* ws_cnt;
-  unsigned* status;  // device status word (bounded waits)
-  const uint8_t* pf;              // optional: bytes to prefetch into L2 for a later call (NULL: none)
-  unsigned long long pf_bytes;    // their size (a multiple of 16)
-  unsigned long long pf_share;    // bytes per CTA (a multiple of 16)
-  int U;   // units = RB * G
-  int P;   // CTAs sharing the units: CTA c owns q units, plus one more if c < r
+  unsigned* status;             // device status word (bounded waits)
+  const uint8_t* pf;            // optional: bytes to prefetch into L2 for a later call (NULL: none)
+  unsigned long long pf_bytes;  // their size (a multiple of 16)
+  unsigned long long pf_share;  // bytes per CTA (a multiple of 16)
+  int U;                        // units = RB * G
+  int P;                        // CTAs sharing the units: CTA c owns q units, plus one more if c < r
   int q, r;
-  int M, N, Np, K, G, RB, S, m0;
+  int M, N, K, G, RB, S, m0;
+  int mts;     // rows of x' per workspace slot: min(M, 8 * NT)
+  int xpitch;  // staged x' row pitch in halves (XS kernels)
 };
 
 __device__ __forceinline__ int cta_first_unit(const GemvParams& p, int c) { return p.q * c + min(c, p.r); }
@@ -54,93 +106,152 @@ __device__ __forceinline__ int cta_of_unit(const GemvParams& p, int u) {
   return u < b ? u / (p.q + 1) : p.r + (u - b) / p.q;
 }
 
-// One shared-memory ring slot per unit: its 2048 B of codes (one TMA bulk copy).  The unit's 64 B of
-// scales and 16 B of zeros are read by the lanes themselves, one unit ahead.
-constexpr int kSlotBytes = 2048;
-constexpr int kSlotStride = 2048;
-#ifndef AWQ_GEMV_RING
-#define AWQ_GEMV_RING 4
-#endif
-constexpr int kRing = AWQ_GEMV_RING;  // units in flight per warp
-__host__ __device__ constexpr int ring_bytes(int nw) { return nw * kRing * kSlotStride; }
-// Activations staged in shared memory (one TMA copy per row after the dependency wait) when they fit.
-constexpr int kXsMaxBytes = 32 * 1024;
-
-// Copies the codes of unit u into a ring slot; completion is counted on `bar`.
-__device__ __forceinline__ void issue_unit(const GemvParams& p, int u, uint8_t* slot, uint64_t* bar) {
-  mbar_arrive_expect_tx(bar, kSlotBytes);
-  bulk_g2s(slot, p.qw + (size_t)u * 128, 2048u, bar);
+// Sub-range of consumer warp w inside the CTA's units [cu0, cu0 + n): first unit and count.
+__device__ __forceinline__ void warp_range(int cu0, int n, int w, int& wu0, int& nw) {
+  const int wq = n / kNW, wr = n % kNW;
+  wu0 = cu0 + wq * w + min(w, wr);
+  nw = wq + (w < wr ? 1 : 0);
 }
 
-// Scale (as float) and zero point of this lane's row in unit u (coalesced across the warp).
-__device__ __forceinline__ void load_meta(const GemvParams& p, int u, int lane, float& sc, uint32_t& z) {
-  sc = __half2float(p.scales[(size_t)u * 32 + lane]);
-  z = (p.qzeros[(size_t)u * 4 + (lane >> 3)] >> (4 * (lane & 7))) & 0xFu;
+// Copies of the c consecutive units from unit u into a ring slot, completion counted on `bar`.  The codes
+// copy (with the barrier's expected byte count) and the scales + zeros copies can come from different lanes,
+// which proceed in parallel; the barrier's phase cannot complete before the arming arrival, so the order in
+// which the lanes' bytes land does not matter.
+__device__ __forceinline__ void issue_codes(const GemvParams& p, int u, int c, uint8_t* slot, uint64_t* bar) {
+  mbar_arrive_expect_tx(bar, (unsigned)c * 2128u);
+  bulk_g2s(slot, p.qw + (size_t)u * kUnitCodeBytes, (unsigned)(c * kUnitCodeBytes), bar);
+}
+__device__ __forceinline__ void issue_meta(const GemvParams& p, int u, int c, uint8_t* slot, uint64_t* bar) {
+  bulk_g2s(slot + kSlotScaleOff, p.scales + (size_t)u * 32, (unsigned)(c * 64), bar);
+  bulk_g2s(slot + kSlotZeroOff, p.qzeros + (size_t)u * 4, (unsigned)(c * 16), bar);
 }
 
-template <int MT>
-__device__ __forceinline__ void unit_dot(const uint4 (&w)[4], float sc, uint32_t z,
-                                         const uint16_t* __restrict__ const (&xg)[MT],
-                                         float (&yacc)[MT]) {
-  const __half2 z1024 = zero_1024(z), nz64 = neg_zero_64(z);
-  const uint32_t magic = magic_1024x2();
-  float part[MT];
+// One unit: y rows (g + 8i, i = 0..3) x columns (8 nt + 2t + j) += S_row * sum_k (q - z) x'.
+// codes / scl / zer: 32-bit shared addresses of the unit's codes, scales and zeros; xb[nt][c]: x' row 8 nt + g
+// (clamped to the pass), channels 128 grp + 32c + 8t .. + 7, as 16 bytes.
+template <int NT>
+__device__ __forceinline__ void unit_mma(uint32_t codes, uint32_t scl, uint32_t zer, int g, int t,
+                                         const uint4 (&xb)[NT][4], float (&yacc)[NT][4][2]) {
+  uint32_t w[2][2][4];  // [half][row g / g + 8][chunk]
 #pragma unroll
-  for (int m = 0; m < MT; ++m) part[m] = 0.f;
-#pragma unroll(MT >= 4 ? 1 : 2)
-  for (int cp = 0; cp < 2; ++cp) {  // pairs of 32-channel chunks
-    __half2 acc[2][MT];
+  for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[0][m] = acc[1][m] = u32_as_h2(0u);
+    for (int cc = 0; cc < 4; ++cc) {
+      w[h][0][cc] = ld_shared_u32(codes + 512 * cc + 16 * (16 * h + g) + 4 * t);
+      w[h][1][cc] = ld_shared_u32(codes + 512 * cc + 16 * (16 * h + g + 8) + 4 * t);
+    }
+  const uint4 zw = ld_shared_v4(zer);  // word i: zero nibbles of rows 8i .. 8i+7
+  float S[4];
 #pragma unroll
-    for (int c2 = 0; c2 < 2; ++c2) {
-      const int c = cp * 2 + c2;
-      const uint32_t ww[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+  for (int i = 0; i < 4; ++i)
+    S[i] = __half2float(__ushort_as_half(ld_shared_u16(scl + 2 * (g + 8 * i))));
+  const uint32_t zws[4] = {zw.x, zw.y, zw.z, zw.w};
+  __half2 zlo[4], zhi[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        __half2 d[4];
-        word_minus_zero(ww[j], z1024, nz64, magic, d);
-        const int a = j & 1;  // two independent accumulator chains
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t z = (zws[i] >> (4 * g)) & 0xFu;
+    zlo[i] = zero_1024(z);
+    zhi[i] = zero_64(z);
+  }
+  const uint32_t m1024 = magic_1024x2(), m64 = magic_64x2();
+  float c[NT][2][2][4];  // [n-tile][half][chunk parity][fragment]
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          const uint4 xv = ldg_cached(xg[m] + c * 32 + j * 8);
-          acc[a][m] = __hfma2(d[0], u32_as_h2(xv.x), acc[a][m]);
-          acc[a][m] = __hfma2(d[1], u32_as_h2(xv.y), acc[a][m]);
-          acc[a][m] = __hfma2(d[2], u32_as_h2(xv.z), acc[a][m]);
-          acc[a][m] = __hfma2(d[3], u32_as_h2(xv.w), acc[a][m]);
-        }
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) c[nt][h][pr][0] = c[nt][h][pr][1] = c[nt][h][pr][2] = c[nt][h][pr][3] = 0.f;
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+    for (int s = 0; s < 2; ++s)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t ua = s ? (w[h][0][cc] >> 8) : w[h][0][cc], ub = s ? (w[h][1][cc] >> 8) : w[h][1][cc];
+        const uint32_t a0 = h2_as_u32(__hsub2(u32_as_h2(and_or<0x000F000Fu>(ua, m1024)), zlo[2 * h]));
+        const uint32_t a1 = h2_as_u32(__hsub2(u32_as_h2(and_or<0x000F000Fu>(ub, m1024)), zlo[2 * h + 1]));
+        const uint32_t a2 = h2_as_u32(__hsub2(u32_as_h2(and_or<0x00F000F0u>(ua, m64)), zhi[2 * h]));
+        const uint32_t a3 = h2_as_u32(__hsub2(u32_as_h2(and_or<0x00F000F0u>(ub, m64)), zhi[2 * h + 1]));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma_16816_f32(c[nt][h][cc & 1], a0, a1, a2, a3, s ? xb[nt][cc].z : xb[nt][cc].x,
+                        s ? xb[nt][cc].w : xb[nt][cc].y);
+      }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      yacc[nt][2 * h][0] = fmaf(S[2 * h], c[nt][h][0][0] + c[nt][h][1][0], yacc[nt][2 * h][0]);
+      yacc[nt][2 * h][1] = fmaf(S[2 * h], c[nt][h][0][1] + c[nt][h][1][1], yacc[nt][2 * h][1]);
+      yacc[nt][2 * h + 1][0] = fmaf(S[2 * h + 1], c[nt][h][0][2] + c[nt][h][1][2], yacc[nt][2 * h + 1][0]);
+      yacc[nt][2 * h + 1][1] = fmaf(S[2 * h + 1], c[nt][h][0][3] + c[nt][h][1][3], yacc[nt][2 * h + 1][1]);
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ void load_xb(const uint16_t* const (&xrow)[NT], int grp, int t, uint4 (&xb)[NT][4]) {
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) xb[nt][cc] = ldg_cached(xrow[nt] + grp * 128 + cc * 32 + t * 8);
+}
+
+// Row block r written directly from a warp's fragments.
+template <int NT>
+__device__ __forceinline__ void store_frag(const GemvParams& p, int r, int g, int t, int mcount,
+                                           const float (&yacc)[NT][4][2]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int n = r * 32 + g + 8 * i;
+    if (n >= p.N) continue;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int m = 8 * nt + 2 * t + j;
+        if (m < mcount) p.y[(size_t)(p.m0 + m) * p.N + n] = __half_as_ushort(__float2half_rn(yacc[nt][i][j]));
+      }
+  }
+}
+
+// A warp's partial of one row block into its shared-memory slot, [m][32 rows].
+template <int NT>
+__device__ __forceinline__ void stash_frag(float* part, int g, int t, int mcount, const float (&yacc)[NT][4][2]) {
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int m = 8 * nt + 2 * t + j;
+      if (m < mcount) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) part[m * 32 + g + 8 * i] = yacc[nt][i][j];
       }
     }
-#pragma unroll
-    for (int m = 0; m < MT; ++m)
-      part[m] += (__low2float(acc[0][m]) + __high2float(acc[0][m])) +
-                 (__low2float(acc[1][m]) + __high2float(acc[1][m]));
-  }
-#pragma unroll
-  for (int m = 0; m < MT; ++m) yacc[m] = fmaf(sc, part[m], yacc[m]);
 }
 
-template <int MT>
-__device__ __forceinline__ void store_y(const GemvParams& p, int rb, int lane, const float (&v)[MT]) {
-  const int n = rb * 32 + lane;
-  const int mcount = min(MT, p.M - p.m0);
-  if (n < p.N) {
+// lane = row of row block r: y[m][32 r + lane] for m < mcount.  (Fixed-size, fully unrolled arrays keep the
+// values in registers: a dynamically indexed array would live in local memory.)
+template <int NT>
+__device__ __forceinline__ void store_row(const GemvParams& p, int r, int lane, int mcount, const float (&v)[8 * NT]) {
+  const int n = r * 32 + lane;
+  if (n >= p.N) return;
 #pragma unroll
-    for (int m = 0; m < MT; ++m)
-      if (m < mcount) p.y[(size_t)(p.m0 + m) * p.N + n] = __half_as_ushort(__float2half_rn(v[m]));
-  }
+  for (int m = 0; m < 8 * NT; ++m)
+    if (m < mcount) p.y[(size_t)(p.m0 + m) * p.N + n] = __half_as_ushort(__float2half_rn(v[m]));
 }
 
-// Sum over the CTAs that share row block r (called by the one warp per CTA that combines r).
-template <int MT>
-__device__ __forceinline__ void cross_cta_combine(const GemvParams& p, int r, int lane, const float (&part)[MT]) {
+// Sum over the CTAs that share row block r (called by the one warp per CTA that combines r; lane = row).
+template <int NT>
+__device__ __forceinline__ void cross_cta_combine(const GemvParams& p, int r, int lane, int mcount,
+                                                  const float (&part)[8 * NT]) {
   const int cf = cta_of_unit(p, r * p.G);
   const int cl = cta_of_unit(p, r * p.G + p.G - 1);
   const int nc = cl - cf + 1;
   const int slot = (int)blockIdx.x - cf;
-  float* base = p.ws_part + (size_t)r * p.S * 32 * MT;  // slots of row block r
+  float* base = p.ws_part + (size_t)r * p.S * 32 * p.mts;  // slots of row block r
 #pragma unroll
-  for (int m = 0; m < MT; ++m) base[(size_t)(slot * MT + m) * 32 + lane] = part[m];
+  for (int m = 0; m < 8 * NT; ++m)
+    if (m < mcount) base[(size_t)(slot * p.mts + m) * 32 + lane] = part[m];
   __threadfence();
   __syncwarp();
   unsigned old = 0;
@@ -148,167 +259,221 @@ __device__ __forceinline__ void cross_cta_combine(const GemvParams& p, int r, in
   old = __shfl_sync(0xFFFFFFFFu, old, 0);
   if (old != (unsigned)(nc - 1)) return;
   __threadfence();
-  float sum[MT];
+  float sum[8 * NT];
 #pragma unroll
-  for (int m = 0; m < MT; ++m) sum[m] = 0.f;
+  for (int m = 0; m < 8 * NT; ++m) sum[m] = 0.f;
   for (int j = 0; j < nc; ++j) {
 #pragma unroll
-    for (int m = 0; m < MT; ++m) sum[m] += (j == slot) ? part[m] : __ldcg(&base[(size_t)(j * MT + m) * 32 + lane]);
+    for (int m = 0; m < 8 * NT; ++m)
+      if (m < mcount) sum[m] += (j == slot) ? part[m] : __ldcg(&base[(size_t)(j * p.mts + m) * 32 + lane]);
   }
-  store_y<MT>(p, r, lane, sum);
+  store_row<NT>(p, r, lane, mcount, sum);
   if (lane == 0) p.ws_cnt[r] = 0u;
 }
 
-#ifndef AWQ_GEMV_MINB_MT1
-#define AWQ_GEMV_MINB_MT1 3
-#endif
-#ifndef AWQ_GEMV_META_AHEAD
-#define AWQ_GEMV_META_AHEAD 2
-#endif
-// NW warps per CTA: 8, 16 or 32.  A 16-warp CTA takes half an SM (64 registers per thread), so the
-// next kernel's CTAs can already be resident beside it; a 32-warp CTA takes a whole SM.
-template <int MT, int NW, bool XS>
-__global__ void __launch_bounds__(NW * 32, (NW == 32 ? 1 : NW == 16 ? 2 : MT == 1 ? AWQ_GEMV_MINB_MT1 : MT == 2 ? 2 : 1))
-    gemv_kernel(const GemvParams p) {
-  extern __shared__ __align__(128) uint8_t ring_smem[];
-  __shared__ __align__(8) uint64_t full[NW][kRing];
+// Dynamic shared memory: [rings][staged x' (XS): rows x xpitch halves][partials: kNW x 2 slots x mcount x 32 fp32].
+__host__ __device__ constexpr int gemv_part_bytes(int rows) { return kNW * 2 * rows * 32 * 4; }
+__host__ __device__ constexpr int gemv_xs_bytes(int rows, int xpitch) { return (rows * xpitch * 2 + 127) / 128 * 128; }
+
+// Producer warp.  Lane L serves CTA slot j = L % kSlotLanes (consumer warp j / kRing, ring index j % kRing):
+// lanes below kSlotLanes issue the slot's codes copy (and arm its barrier), lanes from kSlotLanes on issue its
+// scales and zeros when there are enough lanes, so the big and small copies of a slot are serviced in
+// parallel.  The warp's slot sequence number sq = 0, 1, ... covers its units [sq * kSU, sq * kSU + kSU); ring
+// index si takes the sequence numbers si, si + kRing, ...  The first use of each slot is issued at once
+// (before any dependency wait), later ones when the consumer has released the slot.
+constexpr int kSlotLanes = kSlots <= 16 ? kSlots : 32;  // lanes that issue codes; kSlots <= 16: one more lane for meta
+static_assert(kSlots <= 32, "one producer warp serves at most 32 slots");
+__device__ __forceinline__ void gemv_producer(const GemvParams& p, uint8_t* ring, uint64_t* full, uint64_t* empty,
+                                              int cu0, int n, int lane) {
+  const bool split = kSlots <= 16;
+  const int j = split ? lane % 16 : lane;
+  const bool does_codes = lane < kSlotLanes, does_meta = split ? (lane >= 16 && j < kSlots) : does_codes;
+  if (j >= kSlots || !(does_codes || does_meta)) return;
+  int wu0, nw;
+  warp_range(cu0, n, j / kRing, wu0, nw);
+  const int si = j % kRing;
+  uint8_t* slot = ring + (size_t)j * kSlotStride;
+  auto issue = [&](int sq) {
+    const int u = wu0 + sq * kSU, c = min(kSU, nw - sq * kSU);
+    if (does_codes) issue_codes(p, u, c, slot, &full[j]);
+    if (does_meta) issue_meta(p, u, c, slot, &full[j]);
+  };
+  int next = si;  // next slot sequence number to issue
+  if (next * kSU < nw) {
+    issue(next);
+    next += kRing;
+  }
+  // Refills once the consumer has released the slot (bounded: on a timeout the lane records it, stops issuing
+  // and drains what it issued).
+  bool ok = true;
+  while (next * kSU < nw) {
+    const int use = next / kRing;  // uses of this slot so far; the consumer's release of use - 1 frees it
+    if (!mbar_wait_backoff(&empty[j], (unsigned)(use - 1) & 1u, p.status)) {
+      ok = false;
+      break;
+    }
+    issue(next);
+    next += kRing;
+  }
+  if (!ok) {  // drain: every copy this lane issued lands before the CTA can exit
+    const int last = next - kRing;
+    if (last >= 0 && last * kSU < nw) mbar_wait(&full[j], (unsigned)(last / kRing) & 1u, p.status);
+  }
+}
+
+template <int NT, bool XS>
+__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t full[kSlots];
+  __shared__ __align__(8) uint64_t empty[kSlots];
   __shared__ __align__(8) uint64_t xbar;
-  __shared__ float s_part[NW][2][MT * 32];
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = p.G;
   const int c = blockIdx.x;
   const int cu0 = cta_first_unit(p, c), n = p.q + (c < p.r ? 1 : 0), cu1 = cu0 + n;
-  const int wq = n / NW, wr = n % NW;  // NW is a power of two
-  const int wu0 = cu0 + wq * warp + min(warp, wr), nw = wq + (warp < wr ? 1 : 0), wu1 = wu0 + nw;
-  const bool active = nw > 0;
-  uint8_t* ring = ring_smem + (size_t)warp * kRing * kSlotStride;
+  const int mcount = min(8 * NT, p.M - p.m0);
+  uint8_t* ring = smem;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + kRingBytes);
+  float* s_part = reinterpret_cast<float*>(smem + kRingBytes + (XS ? gemv_xs_bytes(mcount, p.xpitch) : 0));
 
-  // Before the dependency wait: only weights.  The warp's whole sub-range goes towards L2, and the
-  // first kRing units into this warp's shared-memory ring.
-  if (XS && threadIdx.x == 0) {
-    mbar_init(&xbar, 1);
-    fence_mbar_init();
+  for (int j = threadIdx.x; j < kSlots; j += kThreads) {
+    mbar_init(&full[j], 1);
+    mbar_init(&empty[j], 1);
   }
-  if (XS) __syncthreads();
-  if (active && lane == 0) {
-#pragma unroll
-    for (int i = 0; i < kRing; ++i) mbar_init(&full[warp][i], 1);
-    fence_mbar_init();
-    const char* base = reinterpret_cast<const char*>(p.qw + (size_t)wu0 * 128);
-    for (int off = 0; off < nw * 2048; off += 32768)
-      prefetch_l2_bulk(base + off, (unsigned)min(32768, nw * 2048 - off));
-    prefetch_l2_bulk(p.scales + (size_t)wu0 * 32, (unsigned)(nw * 64));
-    prefetch_l2_bulk(p.qzeros + (size_t)wu0 * 4, (unsigned)(nw * 16));
-    for (int i = 0; i < kRing && i < nw; ++i) issue_unit(p, wu0 + i, ring + i * kSlotStride, &full[warp][i]);
+  if (XS && threadIdx.x == 0) mbar_init(&xbar, 1);
+  fence_mbar_init();
+  __syncthreads();
+
+  if (warp == kNW) {  // ---------------------------------------------------------------- producer warp
+    // L2 prefetch of a later call's weights (a caller's hint), spread over the CTAs; weights only.
+    if (p.pf != nullptr && p.m0 == 0 && lane == 31) {
+      const unsigned long long a = (unsigned long long)c * p.pf_share;
+      const unsigned long long e = a + p.pf_share < p.pf_bytes ? a + p.pf_share : p.pf_bytes;
+      for (unsigned long long o = a; o < e; o += 32768ull)
+        prefetch_l2_bulk(p.pf + o, (unsigned)(e - o < 32768ull ? e - o : 32768ull));
+    }
+    gemv_producer(p, ring, full, empty, cu0, n, lane);
+    return;
   }
-  // L2 prefetch of a later call's weights (a caller's hint), spread over the CTAs; weights only.
-  if (p.pf != nullptr && p.m0 == 0 && threadIdx.x == (NW - 1) * 32) {
-    const unsigned long long a = (unsigned long long)c * p.pf_share;
-    const unsigned long long e = a + p.pf_share < p.pf_bytes ? a + p.pf_share : p.pf_bytes;
-    for (unsigned long long o = a; o < e; o += 32768ull)
-      prefetch_l2_bulk(p.pf + o, (unsigned)(e - o < 32768ull ? e - o : 32768ull));
+
+  // ------------------------------------------------------------------------------------ consumer warps
+  const int g4 = lane >> 2, t4 = lane & 3;
+  int wu0, nw;
+  warp_range(cu0, n, warp, wu0, nw);
+  const int wu1 = wu0 + nw;
+  const bool active = nw > 0;
+  const uint32_t ring_addr = smem_u32(ring) + (uint32_t)(warp * kRing * kSlotStride);
+  const uint32_t empty_addr = smem_u32(&empty[warp * kRing]);
+#if AWQ_GEMV_L2_PREFETCH
+  // Before the dependency wait the consumers are idle: each asks for its whole range of codes (32 KB per
+  // lane, lanes in parallel) and of scales and zeros to be brought towards L2, so HBM streams at full rate
+  // from the kernel's start and the producer's ring copies mostly hit L2.
+  if (active) {
+    const int chunks = (nw * kUnitCodeBytes + 32767) / 32768;
+    for (int ch = lane; ch < chunks; ch += 30) {
+      const int off = ch * 32768;
+      prefetch_l2_bulk(p.qw + (size_t)wu0 * kUnitCodeBytes + off, (unsigned)min(32768, nw * kUnitCodeBytes - off));
+    }
+    if (lane == 30) prefetch_l2_bulk(p.scales + (size_t)wu0 * 32, (unsigned)(nw * 64));
+    if (lane == 31) prefetch_l2_bulk(p.qzeros + (size_t)wu0 * 4, (unsigned)(nw * 16));
   }
-  __syncwarp();
-  float sc = 0.f, sc1 = 0.f;
-  uint32_t z = 0u, z1 = 0u;
-  if (active) load_meta(p, wu0, lane, sc, z);  // weights only: no dependency on earlier kernels
-  if (AWQ_GEMV_META_AHEAD == 2 && nw > 1) load_meta(p, wu0 + 1, lane, sc1, z1);
+#endif
   pdl_wait_prior_grids();  // activations, outputs and workspace follow the stream order
 
-  const int mcount = min(MT, p.M - p.m0);
-  const uint16_t* xrow[MT];
-  if (XS) {  // x' rows of this pass -> shared memory, one bulk copy per row
-    uint16_t* xs = reinterpret_cast<uint16_t*>(ring_smem + ring_bytes(NW));
+  const uint16_t* xrow[NT];  // this lane's B column (row 8 nt + g4 of the pass, clamped) per n-tile
+  if (XS) {  // x' rows of this pass -> shared memory, one bulk copy per row (padded pitch)
     if (threadIdx.x == 0) {
       mbar_arrive_expect_tx(&xbar, (unsigned)(mcount * p.K * 2));
-      for (int m = 0; m < mcount; ++m) bulk_g2s(xs + m * p.K, p.x + (size_t)(p.m0 + m) * p.K, (unsigned)(p.K * 2), &xbar);
+      for (int m = 0; m < mcount; ++m)
+        bulk_g2s(xs + m * p.xpitch, p.x + (size_t)(p.m0 + m) * p.K, (unsigned)(p.K * 2), &xbar);
     }
 #pragma unroll
-    for (int m = 0; m < MT; ++m) xrow[m] = xs + min(m, mcount - 1) * p.K;
+    for (int nt = 0; nt < NT; ++nt) xrow[nt] = xs + min(8 * nt + g4, mcount - 1) * p.xpitch;
   } else {
 #pragma unroll
-    for (int m = 0; m < MT; ++m) xrow[m] = p.x + (size_t)(p.m0 + min(m, mcount - 1)) * p.K;
+    for (int nt = 0; nt < NT; ++nt) xrow[nt] = p.x + (size_t)(p.m0 + min(8 * nt + g4, mcount - 1)) * p.K;
   }
-  const int rb_f = active ? wu0 / G : -1;  // the only division of the main path
+  const int rb_f = active ? wu0 / G : -1;
   const int g0 = active ? wu0 - rb_f * G : 0;
+  const int rb_l = active ? (wu1 - 1) / G : -1;  // the warp's last row block
 
   bool ok = true;
   if (XS && active) ok = __all_sync(0xFFFFFFFFu, mbar_wait_backoff(&xbar, 0u, p.status));
-  int rb = rb_f, g = g0, rb_l = rb_f;
+  uint4 xb[NT][4];
+  if (!XS && active) load_xb<NT>(xrow, g0, t4, xb);
+  int rb = rb_f, g = g0;
   int t = 0;  // units of this warp consumed so far
   while (t < nw && ok) {  // segments: the units of one row block inside this warp's range
     const int seg = min(nw - t, G - g);
     const bool whole = (g == 0) && (seg == G);
-    float yacc[MT];
+    float yacc[NT][4][2];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) yacc[m] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) yacc[nt][i][0] = yacc[nt][i][1] = 0.f;
     for (int i = 0; i < seg; ++i, ++t) {
-      const int si = t & (kRing - 1);
-      uint8_t* slot = ring + si * kSlotStride;
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait_backoff(&full[warp][si], (unsigned)(t / kRing) & 1u, p.status));
-      if (!ok) break;  // warp-uniform
-      float scn = 0.f;
-      uint32_t zn = 0u;
-      // scale and zero of a later unit: the next one, or the one after it (two in flight)
-      if (t + AWQ_GEMV_META_AHEAD < nw) load_meta(p, wu0 + t + AWQ_GEMV_META_AHEAD, lane, scn, zn);
-      uint4 w[4];
+      const int sq = t / kSU, ui = t & (kSU - 1);  // slot sequence number and unit within the slot
+      const int si = sq & (kRing - 1);
+      const uint32_t slot = ring_addr + (uint32_t)(si * kSlotStride);
+      uint4 xcur[NT][4];
+      if (XS) {  // B fragments from the staged x'
+        load_xb<NT>(xrow, g + i, t4, xcur);
+      } else {  // loaded one unit ahead from global memory; start the next unit's loads
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) w[cc] = *reinterpret_cast<const uint4*>(slot + cc * 512 + lane * 16);
-      const uint16_t* xg[MT];
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int m = 0; m < MT; ++m) xg[m] = xrow[m] + (g + i) * 128;
-      unit_dot<MT>(w, sc, z, xg, yacc);
-      __syncwarp();  // every lane has consumed the slot
-      if (lane == 0 && t + kRing < nw) {
-        fence_proxy_async_smem();  // our generic reads of the slot before the async-proxy refill
-        issue_unit(p, wu0 + t + kRing, slot, &full[warp][si]);
+          for (int cc = 0; cc < 4; ++cc) xcur[nt][cc] = xb[nt][cc];
+        if (t + 1 < nw) load_xb<NT>(xrow, (g + i + 1 == G) ? 0 : g + i + 1, t4, xb);
       }
-      if (AWQ_GEMV_META_AHEAD == 2) {
-        sc = sc1;
-        z = z1;
-        sc1 = scn;
-        z1 = zn;
-      } else {
-        sc = scn;
-        z = zn;
+      if (ui == 0) {  // first unit of the slot: wait for its copies
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait_backoff(&full[warp * kRing + si], (unsigned)(sq / kRing) & 1u, p.status));
+        if (!ok) break;  // warp-uniform
+      }
+      unit_mma<NT>(slot + (uint32_t)(ui * kUnitCodeBytes), slot + (uint32_t)(kSlotScaleOff + ui * 64),
+                   slot + (uint32_t)(kSlotZeroOff + ui * 16), g4, t4, xcur, yacc);
+      if (ui == kSU - 1 || t == nw - 1) {  // last unit of the slot: every lane has read it; release it
+        __syncwarp();
+        if (lane == 0) mbar_arrive_addr(empty_addr + 8u * (uint32_t)si);
       }
     }
     if (!ok) break;
     if (whole) {
-      store_y<MT>(p, rb, lane, yacc);
+      store_frag<NT>(p, rb, g4, t4, mcount, yacc);
     } else {
-      const int slot = (rb == rb_f) ? 0 : 1;
-#pragma unroll
-      for (int m = 0; m < MT; ++m) s_part[warp][slot][m * 32 + lane] = yacc[m];
+      const int sl = (rb == rb_f) ? 0 : 1;
+      stash_frag<NT>(s_part + (size_t)(warp * 2 + sl) * mcount * 32, g4, t4, mcount, yacc);
     }
-    rb_l = rb;
     ++rb;
     g = 0;
   }
-  if (!ok && lane == 0) {  // give up: wait (bounded) for this warp's copies still in flight
-    for (int j = t; j < nw && j < t + kRing; ++j)
-      mbar_wait(&full[warp][j & (kRing - 1)], (unsigned)(j / kRing) & 1u, p.status);
-  }
-  __syncthreads();
-  if (!active || !ok) return;
-
-  // A split row block r is combined by the warp holding its first unit inside this CTA.
+  // A consumer that gave up leaves the producer's remaining refills unreleased; the producer's bounded
+  // waits run out and it drains its own copies.
+  if (XS && threadIdx.x == 0 && !mbar_try_wait(&xbar, 0u)) mbar_wait(&xbar, 0u, p.status);  // x' copy landed
+  named_barrier_sync(1, kNW * 32);  // consumer warps only: their partials are in shared memory
+  if (!active) return;
+  // A split row block r is combined by the warp holding its first unit inside this CTA.  This runs
+  // whether or not a wait gave up, so that every counter returns to zero.
+  const int wq = n / kNW, wr = n % kNW;
+  // The partial of warp j for row block r sits in its slot 0 when r is warp j's first row block, else in slot 1.
+  // All warps' loads are issued together (unrolled, predicated), so the reduction costs one load latency.
   auto combine = [&](int r) {
     const int a = max(r * G, cu0), b = min((r + 1) * G, cu1);
-    float sum[MT];
+    float sum[8 * NT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) sum[m] = 0.f;
-    for (int j = warp; j < NW; ++j) {
+    for (int m = 0; m < 8 * NT; ++m) sum[m] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kNW; ++j) {
       const int j0 = cu0 + wq * j + min(j, wr), jn = wq + (j < wr ? 1 : 0);
-      if (j0 >= b) break;
-      if (jn == 0) continue;
-      const int slot = (j0 >= r * G) ? 0 : 1;  // r is warp j's first row block iff it starts at or before j0
+      // warp j holds units [j0, j0 + jn); it has a partial of r iff that range meets [a, b)
+      const bool has = jn > 0 && j0 < b && j0 + jn > a;
+      const float* src = s_part + (size_t)(j * 2 + ((j0 >= r * G) ? 0 : 1)) * mcount * 32 + lane;
 #pragma unroll
-      for (int m = 0; m < MT; ++m) sum[m] += s_part[j][slot][m * 32 + lane];
+      for (int m = 0; m < 8 * NT; ++m)
+        if (has && m < mcount) sum[m] += src[m * 32];
     }
-    if (a == r * G && b == (r + 1) * G) store_y<MT>(p, r, lane, sum);
-    else cross_cta_combine<MT>(p, r, lane, sum);
+    if (a == r * G && b == (r + 1) * G) store_row<NT>(p, r, lane, mcount, sum);
+    else cross_cta_combine<NT>(p, r, lane, mcount, sum);
   };
   const bool whole_f = (g0 == 0) && (nw >= G);
   const bool owner_f = (g0 == 0) || (wu0 == cu0);
@@ -318,145 +483,68 @@ __global__ void __launch_bounds__(NW * 32, (NW == 32 ? 1 : NW == 16 ? 2 : MT == 
 
 // ------------------------------------------------------------------------------------------ host
 #ifndef AWQ_GEMV_CTAS_PER_SM
-#define AWQ_GEMV_CTAS_PER_SM 4
-#endif
-#ifndef AWQ_GEMV_WHOLE_RB_MAX_UNITS
-#define AWQ_GEMV_WHOLE_RB_MAX_UNITS 48
-#endif
-#ifndef AWQ_GEMV_BIG_CTA_WARPS  // warps of the one-row-block-per-CTA plan: 16 or 32
-#define AWQ_GEMV_BIG_CTA_WARPS 16
-#endif
-#ifndef AWQ_GEMV_STAGE_X  // stage activations in shared memory when they fit
-#define AWQ_GEMV_STAGE_X 1
+#define AWQ_GEMV_CTAS_PER_SM 1
 #endif
 
 namespace {
 
-int pick_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
-
-template <int MT, int NW, bool XS>
+template <int NT, bool XS>
 bool gemv_smem_attr() {
   static bool done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(gemv_kernel<MT, NW, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ring_bytes(NW) + (XS ? kXsMaxBytes : 0)) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemv_kernel<NT, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) !=
+        cudaSuccess)
       return false;
     done[dev] = true;
   }
   return true;
 }
 
-#ifndef AWQ_GEMV_OCC_EXACT
-#define AWQ_GEMV_OCC_EXACT 1
-#endif
-// 8-warp CTAs of one launch resident per SM (at most AWQ_GEMV_CTAS_PER_SM), for the shared memory the
-// launch really uses: the rings plus xs_bytes of staged activations (0: not staged).
-template <int MT>
-int resident_ctas_mt(int xs_bytes) {
-  static int cached[64][kXsMaxBytes / 256 + 1] = {{0}};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  if (!AWQ_GEMV_OCC_EXACT) xs_bytes = kXsMaxBytes;  // sized for the largest staging
-  const int i = (xs_bytes + 255) / 256;
-  if (cached[dev][i] == 0) {
-    int occ = 0;
-    cudaError_t e;
-    if (xs_bytes > 0) {
-      gemv_smem_attr<MT, 8, true>();
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<MT, 8, true>, 8 * 32,
-                                                        ring_bytes(8) + i * 256);
-    } else {
-      gemv_smem_attr<MT, 8, false>();
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<MT, 8, false>, 8 * 32, ring_bytes(8));
-    }
-    if (e != cudaSuccess || occ < 1) occ = 1;
-    cached[dev][i] = occ < AWQ_GEMV_CTAS_PER_SM ? occ : AWQ_GEMV_CTAS_PER_SM;
-  }
-  return cached[dev][i];
-}
-
-int resident_ctas(int MT, int xs_bytes) {
-  switch (MT) {
-    case 1: return resident_ctas_mt<1>(xs_bytes);
-    default: return resident_ctas_mt<2>(xs_bytes);
-  }
-}
-int resident_ctas_big(int MT) {  // MT 4 and 8 never stage activations
-  static int cached[64][2] = {{0}};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  const int i = MT == 4 ? 0 : 1;
-  if (cached[dev][i] == 0) {
-    int occ = 0;
-    cudaError_t e;
-    if (MT == 4) {
-      gemv_smem_attr<4, 8, false>();
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<4, 8, false>, 256, ring_bytes(8));
-    } else {
-      gemv_smem_attr<8, 8, false>();
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv_kernel<8, 8, false>, 256, ring_bytes(8));
-    }
-    if (e != cudaSuccess || occ < 1) occ = 1;
-    cached[dev][i] = occ < AWQ_GEMV_CTAS_PER_SM ? occ : AWQ_GEMV_CTAS_PER_SM;
-  }
-  return cached[dev][i];
-}
-
 struct GemvPlan {
-  int MT, NW, RB, G, S, Np, P;
-  bool xs;  // activations staged in shared memory
-  int U, q, r;
+  int NT, mts, RB, G, U, P, q, r, S;
+  bool xs;     // x' staged in shared memory
+  int xpitch;  // its row pitch in halves
   size_t part_bytes;
 };
 
-// Three shapes of work, chosen so that all CTAs of a launch are resident at once:
-//  - at most one row block per SM (and M <= 2): one 16-warp CTA per row block; its warps split the
-//    row block's groups and combine in shared memory -- no partial sum leaves a CTA;
-//  - short row blocks (G <= 48) that fit the 8-warp CTAs resident on all SMs: one 8-warp CTA per row
-//    block, likewise self-contained;
-//  - otherwise the units are spread evenly over all resident 8-warp CTAs and the row blocks cut by CTA
-//    boundaries are combined in the workspace.
+// Two shapes of work, at most AWQ_GEMV_CTAS_PER_SM CTAs per SM:
+//  - at most that many row blocks: one CTA per row block; its warps split the row block's groups and
+//    combine in shared memory -- no partial sum leaves a CTA;
+//  - otherwise the units are spread evenly over the CTAs and the row blocks cut by CTA boundaries are
+//    combined in the workspace.
 GemvPlan plan_gemv(int M, int N, int K) {
   GemvPlan pl{};
-  pl.MT = pick_mt(M);
-  pl.Np = (N + 31) / 32 * 32;
-  pl.RB = pl.Np / 32;
+  pl.NT = M <= 8 ? 1 : 2;
+  pl.mts = M < 8 * pl.NT ? M : 8 * pl.NT;
+  pl.RB = (N + 31) / 32;
   pl.G = K / 128;
   pl.U = pl.RB * pl.G;
-  const int sms = num_sms();
+  pl.xpitch = K + kXPad;
+  pl.xs = pl.mts * pl.xpitch * 2 <= kXsMaxBytes &&
+          kRingBytes + gemv_xs_bytes(pl.mts, pl.xpitch) + gemv_part_bytes(pl.mts) <= kMaxDynSmem;
+  const int p_max = num_sms() * AWQ_GEMV_CTAS_PER_SM;
   pl.S = 1;
   pl.part_bytes = 0;
-  if (pl.MT <= 2 && pl.RB <= sms) {
-    pl.NW = AWQ_GEMV_BIG_CTA_WARPS;
+  if (pl.RB <= p_max) {
     pl.P = pl.RB;
   } else {
-    pl.NW = 8;
-    const int xs_bytes = (AWQ_GEMV_STAGE_X && pl.MT <= 2 && pl.MT * K * 2 <= kXsMaxBytes) ? pl.MT * K * 2 : 0;
-    int p_bal = sms * (pl.MT <= 2 ? resident_ctas(pl.MT, xs_bytes) : resident_ctas_big(pl.MT));
-    const int by_units = pl.U / 8 > 0 ? pl.U / 8 : 1;
-    if (p_bal > by_units) p_bal = by_units;
-    if (pl.RB <= p_bal && pl.G <= AWQ_GEMV_WHOLE_RB_MAX_UNITS) {
-      pl.P = pl.RB;
-    } else {
-      pl.P = p_bal;
-      const int L = pl.U / pl.P;  // >= 1 units per CTA
-      pl.S = pl.G >= 2 ? (pl.G - 2) / L + 2 : 1;
-      pl.part_bytes = (size_t)pl.RB * pl.S * 32 * pl.MT * sizeof(float);
-    }
+    pl.P = p_max;
+    const int L = pl.U / pl.P;  // >= 1 units per CTA
+    pl.S = pl.G >= 2 ? (pl.G - 2) / L + 2 : 1;
+    pl.part_bytes = (size_t)pl.RB * pl.S * 32 * pl.mts * sizeof(float);
   }
   pl.q = pl.U / pl.P;
   pl.r = pl.U % pl.P;
-  pl.xs = AWQ_GEMV_STAGE_X && pl.MT <= 2 && pl.MT * K * 2 <= kXsMaxBytes;
   return pl;
 }
 
-template <int MT, int NW, bool XS>
-cudaError_t launch_mt(const GemvParams& p, cudaStream_t st) {
-  if (!gemv_smem_attr<MT, NW, XS>()) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)ring_bytes(NW) + (XS ? (size_t)MT * p.K * 2 : 0);
-  return launch_pdl(gemv_kernel<MT, NW, XS>, dim3((unsigned)p.P), dim3(NW * 32), smem, st, p);
+template <int NT, bool XS>
+cudaError_t launch_nt(const GemvParams& p, int mcount, cudaStream_t st) {
+  if (!gemv_smem_attr<NT, XS>()) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)kRingBytes + (XS ? gemv_xs_bytes(mcount, p.xpitch) : 0) + gemv_part_bytes(mcount);
+  return launch_pdl(gemv_kernel<NT, XS>, dim3((unsigned)p.P), dim3(kThreads), smem, st, p);
 }
 
 }  // namespace
@@ -475,8 +563,8 @@ awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
     return AWQ_ERR_WORKSPACE;
   GemvParams p;
   p.x = x;
-  p.qw = reinterpret_cast<const uint4*>(qw);
-  p.scales = reinterpret_cast<const __half*>(scales);
+  p.qw = reinterpret_cast<const uint8_t*>(qw);
+  p.scales = scales;
   p.qzeros = qzeros;
   p.y = y;
   p.ws_cnt = static_cast<unsigned*>(ws);
@@ -491,28 +579,20 @@ awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
   p.r = pl.r;
   p.M = M;
   p.N = N;
-  p.Np = pl.Np;
   p.K = K;
   p.G = pl.G;
   p.RB = pl.RB;
   p.S = pl.S;
-  // passes of MT rows run one after the other on the stream and share the workspace
-  for (int m0 = 0; m0 < M; m0 += pl.MT) {
+  p.mts = pl.mts;
+  p.xpitch = pl.xpitch;
+  // passes of 8 * NT rows run one after the other on the stream and share the workspace
+  const int rows = 8 * pl.NT;
+  for (int m0 = 0; m0 < M; m0 += rows) {
     p.m0 = m0;
+    const int mcount = M - m0 < rows ? M - m0 : rows;
     cudaError_t e;
-    if (pl.NW == 16 || pl.NW == 32) {
-      constexpr int BW = AWQ_GEMV_BIG_CTA_WARPS;
-      static_assert(ring_bytes(BW) + kXsMaxBytes <= 227 * 1024, "GEMV shared memory over the per-CTA limit");
-      if (pl.MT == 1) e = pl.xs ? launch_mt<1, BW, true>(p, st) : launch_mt<1, BW, false>(p, st);
-      else e = pl.xs ? launch_mt<2, BW, true>(p, st) : launch_mt<2, BW, false>(p, st);
-    } else {
-      switch (pl.MT) {
-        case 1: e = pl.xs ? launch_mt<1, 8, true>(p, st) : launch_mt<1, 8, false>(p, st); break;
-        case 2: e = pl.xs ? launch_mt<2, 8, true>(p, st) : launch_mt<2, 8, false>(p, st); break;
-        case 4: e = launch_mt<4, 8, false>(p, st); break;
-        default: e = launch_mt<8, 8, false>(p, st); break;
-      }
-    }
+    if (pl.NT == 1) e = pl.xs ? launch_nt<1, true>(p, mcount, st) : launch_nt<1, false>(p, mcount, st);
+    else e = pl.xs ? launch_nt<2, true>(p, mcount, st) : launch_nt<2, false>(p, mcount, st);
     if (e != cudaSuccess) return AWQ_ERR_CUDA;
   }
   return AWQ_OK;

@@ -9,8 +9,8 @@
 // The host code below never passes the array's name to a kernel (in host code it is only a stand-in);
 // it looks up the array's device address once per device with cudaGetSymbolAddress and passes that.
 // The first call on each device performs this lookup, so make that first call before any stream
-// capture.  Every call shares the one array and keeps the last call's contents, so each call clears
-// the counters that must start at zero (cudaMemsetAsync, no allocation).  Calls on one device that
+// capture.  Every call shares the one array and keeps the last call's contents, so each call whose
+// plan uses the scratch clears the counters that must start at zero (cudaMemsetAsync, no allocation).  Calls on one device that
 // overlap on the GPU (for example, issued on two streams) race on the array; the caller must order
 // them.  Each device has its own copy of the array.
 #include "common.cuh"
@@ -42,12 +42,15 @@ extern "C" awq_status w4a16_gemv_noalloc(const uint16_t* d_x, const uint32_t* d_
   using namespace awq;
   awq_status st = check_linear(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g);
   if (st != AWQ_OK) return st;
-  if (gemv_workspace_bytes(M, N, K) > kNoAllocScratchBytes) return AWQ_ERR_WORKSPACE;
+  const size_t need = gemv_workspace_bytes(M, N, K);
+  if (need > kNoAllocScratchBytes) return AWQ_ERR_WORKSPACE;
   void* scratch = noalloc_scratch_address();
   if (scratch == nullptr) return AWQ_ERR_CUDA;
   unsigned* status = device_status_ptr();
   if (status == nullptr) return AWQ_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, kWorkspaceCounterBytes, s) != cudaSuccess) return AWQ_ERR_CUDA;
+  // Only a split plan touches the scratch; a plan without split row blocks needs no clearing (and a
+  // memset between two GEMVs would keep the second from overlapping the first).
+  if (need > 0 && cudaMemsetAsync(scratch, 0, kWorkspaceCounterBytes, s) != cudaSuccess) return AWQ_ERR_CUDA;
   return gemv_launch(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, scratch, kNoAllocScratchBytes, status, s);
 }

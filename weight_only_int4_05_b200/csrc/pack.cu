@@ -8,65 +8,73 @@
 //   w' = W*s; sc32 = max((max-min)/15, 1e-5); S = float(fp16(sc32)); z = clamp(rint(-min/S), 0, 15);
 //   q = clamp(rint(w'/S) + z, 0, 15).
 //
-// One CTA per packed unit (32-row block rb, group g): 8 warps x 4 rows, lane l holds channels
-// 4l..4l+3 of the group (one 8-byte load per row), min/max by warp shuffles, codes assembled into the
-// nibble order of the layout with one shuffle, and the 2 KB unit written from shared memory with
-// coalesced 16-byte stores (the unit's 32 scales and 4 zero words are contiguous too).  The kernel streams 2 bytes in and 0.52 bytes out per weight.
+// One CTA per run of kPackGroups units of one row block (the units (rb, g0 .. g0+3) are consecutive in all
+// three packed arrays).  Each half-warp takes one (row, group): lane h of the half holds channels 8h..8h+7
+// (one 16-byte load), which are exactly the 8 codes of one packed word, so no lane exchange is needed to
+// assemble it.  Min and max come from four shuffles inside the half-warp.  The units are assembled in shared
+// memory and written with coalesced 16-byte stores.  The kernel streams 2 bytes in and 0.52 bytes out per
+// weight.
 #include "common.cuh"
 #include "internal.h"
 
 namespace awq {
 
+constexpr int kPackGroups = 4;  // units per CTA
+
 __device__ __forceinline__ float clamp015(float v) { return fminf(fmaxf(v, 0.0f), 15.0f); }
+__device__ __forceinline__ float h2f_bits(uint32_t bits) { return __half2float(__ushort_as_half((unsigned short)bits)); }
 
 __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W, const __half* __restrict__ s,
-                                                    int N, int K, int Np, int G, uint4* __restrict__ qw,
+                                                    int N, int K, int G, uint8_t* __restrict__ qw,
                                                     uint16_t* __restrict__ scales, uint32_t* __restrict__ qz) {
-  pdl_launch_dependents();
-  __shared__ __align__(16) uint32_t s_words[512];
-  __shared__ uint16_t s_sc[32];
-  __shared__ uint32_t s_z[32];
-  const int g = blockIdx.x, rb = blockIdx.y;
+  // No griddepcontrol.launch_dependents here: the linear kernels read packed weights before their own
+  // dependency wait, so a kernel launched after this one must not start until every packed byte is
+  // written.  Without an explicit trigger the dependents start only when this grid has completed.
+  __shared__ __align__(16) uint32_t s_words[kPackGroups * 512];
+  __shared__ __align__(16) uint16_t s_sc[kPackGroups * 32];
+  __shared__ uint8_t s_zb[kPackGroups * 32];
+  const int rb = blockIdx.x, g0 = blockIdx.y * kPackGroups;
+  const int ng = min(kPackGroups, G - g0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int k0 = g * 128 + lane * 4;
+  const int half = lane >> 4, hl = lane & 15;
   pdl_wait_prior_grids();
 
-  float sv[4] = {1.f, 1.f, 1.f, 1.f};
-  if (s != nullptr) {
-    const uint2 sr = *reinterpret_cast<const uint2*>(s + k0);
-    sv[0] = __half2float(__ushort_as_half((unsigned short)(sr.x & 0xFFFF)));
-    sv[1] = __half2float(__ushort_as_half((unsigned short)(sr.x >> 16)));
-    sv[2] = __half2float(__ushort_as_half((unsigned short)(sr.y & 0xFFFF)));
-    sv[3] = __half2float(__ushort_as_half((unsigned short)(sr.y >> 16)));
+  // rows 4 * warp + 2 * i + half (i = 0, 1) of the row block; all loads first
+  uint4 raw[2][kPackGroups];
+  uint4 sraw[kPackGroups];
+#pragma unroll
+  for (int gi = 0; gi < kPackGroups; ++gi) {
+    const int k0 = (g0 + gi) * 128 + 8 * hl;
+    sraw[gi] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);  // s = 1
+    if (gi < ng && s != nullptr) sraw[gi] = *reinterpret_cast<const uint4*>(s + k0);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int n = rb * 32 + 4 * warp + 2 * i + half;
+      raw[i][gi] = (gi < ng && n < N) ? *reinterpret_cast<const uint4*>(W + (size_t)n * K + k0) : make_uint4(0u, 0u, 0u, 0u);
+    }
   }
-  uint2 raw[4];
+  // nibble position of channel offset e in a word: even e -> e/2, odd e -> 4 + e/2
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int n = rb * 32 + warp * 4 + i;
-    raw[i] = n < N ? *reinterpret_cast<const uint2*>(W + (size_t)n * K + k0) : make_uint2(0u, 0u);
-  }
-  // nibble position of this lane's 4 channels (offsets e = 4*(lane&1) + i inside an 8-channel word):
-  // even e -> e/2, odd e -> 4 + e/2
-  const int odd = lane & 1;
-  const int pos0 = odd ? 2 : 0, pos1 = odd ? 6 : 4, pos2 = odd ? 3 : 1, pos3 = odd ? 7 : 5;
-
+  for (int gi = 0; gi < kPackGroups; ++gi) {
+    if (gi >= ng) break;  // CTA-uniform
+    const uint32_t sw[4] = {sraw[gi].x, sraw[gi].y, sraw[gi].z, sraw[gi].w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = warp * 4 + i;
-    const int n = rb * 32 + r;
-    uint32_t word = 0u;
-    uint16_t sch_bits = 0;
-    uint32_t zi = 0u;
-    if (n < N) {  // warp-uniform
-      float wp[4];
-      wp[0] = __fmul_rn(__half2float(__ushort_as_half((unsigned short)(raw[i].x & 0xFFFF))), sv[0]);
-      wp[1] = __fmul_rn(__half2float(__ushort_as_half((unsigned short)(raw[i].x >> 16))), sv[1]);
-      wp[2] = __fmul_rn(__half2float(__ushort_as_half((unsigned short)(raw[i].y & 0xFFFF))), sv[2]);
-      wp[3] = __fmul_rn(__half2float(__ushort_as_half((unsigned short)(raw[i].y >> 16))), sv[3]);
-      float mn = fminf(fminf(wp[0], wp[1]), fminf(wp[2], wp[3]));
-      float mx = fmaxf(fmaxf(wp[0], wp[1]), fmaxf(wp[2], wp[3]));
+    for (int i = 0; i < 2; ++i) {
+      const int r = 4 * warp + 2 * i + half;
+      const bool valid = rb * 32 + r < N;
+      const uint32_t ww[4] = {raw[i][gi].x, raw[i][gi].y, raw[i][gi].z, raw[i][gi].w};
+      float wp[8];
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
+      for (int e = 0; e < 8; ++e)
+        wp[e] = __fmul_rn(h2f_bits(ww[e >> 1] >> (16 * (e & 1))), h2f_bits(sw[e >> 1] >> (16 * (e & 1))));
+      float mn = wp[0], mx = wp[0];
+#pragma unroll
+      for (int e = 1; e < 8; ++e) {
+        mn = fminf(mn, wp[e]);
+        mx = fmaxf(mx, wp[e]);
+      }
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) {  // inside the half-warp
         mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
         mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
       }
@@ -74,41 +82,41 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
       const __half sch = __float2half_rn(sc32);
       const float S = __half2float(sch);
       const float zf = clamp015(rintf(__fdiv_rn(-mn, S)));
-      zi = (uint32_t)(int)zf;
-      uint32_t c[4];
+      uint32_t word = 0u;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) c[e] = (uint32_t)(int)clamp015(__fadd_rn(rintf(__fdiv_rn(wp[e], S)), zf));
-      const uint32_t part = (c[0] << (4 * pos0)) | (c[1] << (4 * pos1)) | (c[2] << (4 * pos2)) |
-                            (c[3] << (4 * pos3));
-      word = part | __shfl_xor_sync(0xFFFFFFFFu, part, 1);
-      sch_bits = __half_as_ushort(sch);
-    }
-    if (!odd) s_words[(lane >> 3) * 128 + r * 4 + ((lane & 7) >> 1)] = word;
-    if (lane == 0) {
-      s_sc[r] = sch_bits;
-      s_z[r] = zi;
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t code = (uint32_t)(int)clamp015(__fadd_rn(rintf(__fdiv_rn(wp[e], S)), zf));
+        word |= code << (4 * ((e & 1) ? 4 + (e >> 1) : (e >> 1)));
+      }
+      // word hl & 3 of row r in the unit's chunk hl >> 2 (chunk = 512 B = 128 words, row = 4 words)
+      s_words[gi * 512 + (hl >> 2) * 128 + r * 4 + (hl & 3)] = valid ? word : 0u;
+      if (hl == 0) {
+        s_sc[gi * 32 + r] = valid ? __half_as_ushort(sch) : (uint16_t)0;
+        s_zb[gi * 32 + r] = valid ? (uint8_t)(int)zf : (uint8_t)0;
+      }
     }
   }
   __syncthreads();
-  if (threadIdx.x < 128)
-    qw[((size_t)rb * G + g) * 128 + threadIdx.x] = reinterpret_cast<const uint4*>(s_words)[threadIdx.x];
-  const size_t unit = (size_t)rb * G + g;  // scales and zeros are unit major
-  if (threadIdx.x < 32) scales[unit * 32 + threadIdx.x] = s_sc[threadIdx.x];
-  if (threadIdx.x < 4) {
+  const size_t u0 = (size_t)rb * G + g0;  // first unit of this CTA; its ng units are consecutive
+  uint4* dst = reinterpret_cast<uint4*>(qw + u0 * 2048);
+  for (int idx = threadIdx.x; idx < ng * 128; idx += 256) dst[idx] = reinterpret_cast<const uint4*>(s_words)[idx];
+  if (threadIdx.x < ng * 4) {
+    reinterpret_cast<uint4*>(scales + u0 * 32)[threadIdx.x] = reinterpret_cast<const uint4*>(s_sc)[threadIdx.x];
     uint32_t zw = 0u;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) zw |= s_z[threadIdx.x * 8 + i] << (4 * i);
-    qz[unit * 4 + threadIdx.x] = zw;
+    for (int i = 0; i < 8; ++i) zw |= (uint32_t)s_zb[threadIdx.x * 8 + i] << (4 * i);
+    qz[u0 * 4 + threadIdx.x] = zw;
   }
+  __threadfence();  // the packed units are performed at device scope before this CTA exits
 }
 
 awq_status pack_launch(const uint16_t* W, const uint16_t* s, int N, int K, uint32_t* qw, uint16_t* scales,
                        uint32_t* qz, cudaStream_t st) {
-  const int Np = (N + 31) / 32 * 32;
+  const int RB = (N + 31) / 32;
   const int G = K / 128;
-  cudaError_t e = launch_pdl(pack_kernel, dim3((unsigned)G, (unsigned)(Np / 32)), dim3(256), 0, st,
-                             reinterpret_cast<const __half*>(W), reinterpret_cast<const __half*>(s), N, K, Np, G,
-                             reinterpret_cast<uint4*>(qw), scales, qz);
+  const dim3 grid((unsigned)RB, (unsigned)((G + kPackGroups - 1) / kPackGroups));  // x: row blocks (no 65535 cap)
+  cudaError_t e = launch_pdl(pack_kernel, grid, dim3(256), 0, st, reinterpret_cast<const __half*>(W),
+                             reinterpret_cast<const __half*>(s), N, K, G, reinterpret_cast<uint8_t*>(qw), scales, qz);
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
