@@ -180,8 +180,10 @@ awq_status w4a16_gemm(const uint16_t* d_x, const uint32_t* d_qweight, const uint
 /* w4a16_gemv_noalloc -- the same computation as w4a16_gemv for callers that cannot allocate device
  * memory (e.g. a plug-in whose host framework owns every allocation, or a serving loop whose memory
  * budget is fixed at start-up).  The pages have no counterpart: this is a deployment convenience.
- * The split-K scratch is a library-owned static device array of 8 MiB per device (held by every GPU
- * that loads the library until exit); sizes whose scratch would exceed it return AWQ_ERR_WORKSPACE.
+ * The split scratch is a library-owned static device array of 512 KiB per device (held by every GPU
+ * that loads the library until exit); sizes whose scratch would exceed it return AWQ_ERR_WORKSPACE.  Most
+ * shapes need no scratch at all (w4a16_workspace_bytes(AWQ_MODE_GEMV, ...) == 0); the array serves the
+ * shapes whose row blocks are split between CTAs.
  * Nothing is allocated: the call clears the array's counters with cudaMemsetAsync and launches the
  * GEMV.  The first call on a device looks up the array's address (cudaGetSymbolAddress); make it
  * before any stream capture.  All calls share the array: calls that overlap on the GPU race. */

@@ -127,3 +127,20 @@ def test_linear_dispatch_matches_selected_mode():
 
 def test_device_status_clean_after_runs():
     assert W4.awq_last_device_status() == 0
+
+
+@pytest.mark.parametrize("N", [4864, 4800])
+@pytest.mark.parametrize("M", [1, 3, 8, 12])
+def test_gemv_split_row_blocks_between_ctas(M, N):
+    """A few row blocks more than SMs (150, 152): the units are spread evenly over the CTAs and the row blocks
+    cut by CTA boundaries are summed in the workspace (deterministic slot order)."""
+    assert W4.w4a16_workspace_bytes(W4.MODE_GEMV, M, N, 4096) > 0
+    case = OracleCase(6, 0, M, N % 7, M, N, 4096)
+    _, xp, pw = run_prep_and_pack(case)
+    y = W4.w4a16_gemv(xp, pw)
+    y2 = W4.w4a16_gemv(xp, pw)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+    ms, ns = sample_pairs(M, N, 1500, seed=N + M)
+    assert_within_tolerance(y.float().cpu().numpy()[ms, ns], case.y_pairs(ms, ns), f"gemv split M={M} N={N}")
+    assert W4.awq_last_device_status() == 0

@@ -33,12 +33,12 @@ def test_wait_gives_up_and_reports_timeout(backoff):
 
 
 def test_split_shapes_after_a_timeout_use_the_cached_workspace():
-    """After a wait ran out, split shapes (cross-CTA GEMV combine at 4096 -> 14336, split-K GEMM at
+    """After a wait ran out, split shapes (cross-CTA GEMV combine at 4096 -> 4864, split-K GEMM at
     14336 -> 4096) still find every counter of the shared workspace at zero and match the oracle."""
     torch.cuda.set_device(0)
     assert W4.awq_selftest_wait_timeout(False) == 1
     assert W4.awq_last_device_status() == 5
-    for (N, K, M, fn, mode) in ((14336, 4096, 1, W4.w4a16_gemv, W4.MODE_GEMV),
+    for (N, K, M, fn, mode) in ((4864, 4096, 1, W4.w4a16_gemv, W4.MODE_GEMV),
                                 (4096, 14336, 8, W4.w4a16_gemm, W4.MODE_GEMM)):
         case = OracleCase(0, 1, 0, 2 if N > K else 3, M, N, K)
         s = W4.awq_act_scale(dev(case.xcal))

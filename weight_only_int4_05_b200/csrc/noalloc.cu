@@ -3,7 +3,7 @@
 // Some callers have no way to hand this library a workspace: a plug-in whose host framework owns every
 // device allocation and exposes no allocator to it, or a serving loop with a device-memory budget
 // fixed at start-up that must not allocate per request.  For them the GEMV's split-K scratch lives in
-// a file-scope __device__ array of kNoAllocScratchBytes, which every GPU that loads this library holds
+// a file-scope __device__ array of kNoAllocScratchBytes (512 KiB), which every GPU that loads this library holds
 // until the process exits.
 //
 // The host code below never passes the array's name to a kernel (in host code it is only a stand-in);
@@ -18,7 +18,7 @@
 
 namespace awq {
 
-constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+constexpr size_t kNoAllocScratchBytes = size_t(512) << 10;  // 512 KiB per device
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
