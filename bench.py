@@ -201,11 +201,15 @@ def summarize_clock_lines(lines):
 class DecodeStack:
     """32 layers x 7 packed linears, inputs x' and outputs y resident in HBM, one CUDA graph per step."""
 
-    def __init__(self, device, seed=0, M=1, layers=LAYERS, inputs_fn=None, prefetch=False, fused=False):
+    def __init__(self, device, seed=0, M=1, layers=LAYERS, inputs_fn=None, prefetch=False, fused=False,
+                 inv_s_fused=False):
         """inputs_fn(layer, linear, M, N, K) -> (W, xcal, x) fp16 device tensors; default: the seeded
         device generator of the synthetic workload.  prefetch: each call passes the next linear's packed
-        weight as an L2 prefetch hint (w4a16_linear_pf).  fused: 4 linears per layer (FUSED_SHAPES)."""
+        weight as an L2 prefetch hint (w4a16_linear_pf).  fused: 4 linears per layer (FUSED_SHAPES).
+        inv_s_fused: the resident activations are the raw x and every call is w4a16_gemv_s(x, s), which
+        divides by the AWQ scale inside the kernel (no separate 1/s pass)."""
         self.prefetch = prefetch
+        self.inv_s_fused = inv_s_fused
         layer_shapes = FUSED_SHAPES if fused else DECODE_SHAPES
         cfg = 6 if fused else 2  # tensor-id namespace of the synthetic inputs
         import torch
@@ -214,6 +218,7 @@ class DecodeStack:
 
         self.W4, self.torch, self.device, self.M = W4, torch, device, M
         self.entries = []  # (packed weight, x' view, y view)
+        self.s_list = []   # AWQ scales (inv_s_fused only)
         shapes = [(li, name, K, N) for li in range(layers) for (name, K, N) in layer_shapes]
         self.h2d_elems = sum(M * K for _, _, K, _ in shapes)
         self.d2h_elems = sum(M * N for _, _, _, N in shapes)
@@ -229,7 +234,11 @@ class DecodeStack:
             s = W4.awq_act_scale(xcal)
             pw = W4.awq_pack(Wt, s)
             xv = self.x_all[xo:xo + M * K].view(M, K)
-            W4.awq_apply_inv_scale(x, s, out=xv)
+            if inv_s_fused:
+                xv.copy_(x)
+                self.s_list.append(s)
+            else:
+                W4.awq_apply_inv_scale(x, s, out=xv)
             yv = self.y_all[yo:yo + M * N].view(M, N)
             self.entries.append((pw, xv, yv, K, N))
             xo += M * K
@@ -250,7 +259,9 @@ class DecodeStack:
     def eager_step(self):
         n = len(self.entries)
         for i, (pw, xv, yv, _, _) in enumerate(self.entries):
-            if self.prefetch:  # the next linear of the step (the first one of the next step at the end)
+            if self.inv_s_fused:
+                self.W4.w4a16_gemv_s(xv, self.s_list[i], pw, out=yv)
+            elif self.prefetch:  # the next linear of the step (the first one of the next step at the end)
                 self.W4.w4a16_linear_pf(xv, pw, self.entries[(i + 1) % n][0], out=yv)
             else:
                 self.W4.w4a16_linear(xv, pw, out=yv)
@@ -272,7 +283,8 @@ class DecodeStack:
         self.graph.replay()
 
     def bytes_per_step(self):
-        return sum(gemv_bytes(self.M, N, K) for _, _, _, K, N in self.entries)
+        extra = sum(2 * K for _, _, _, K, _ in self.entries) if self.inv_s_fused else 0  # the scale vectors
+        return sum(gemv_bytes(self.M, N, K) for _, _, _, K, N in self.entries) + extra
 
 
 class PrefillGemm:
@@ -656,6 +668,20 @@ def run_gpu(args):
     del fstack
     torch.cuda.empty_cache()
 
+    # ---- the plain stack with the AWQ 1/s fused into every GEMV (raw x and s in, no separate scaling pass)
+    sstack = DecodeStack(device, inv_s_fused=True)
+    sstack.capture()
+    s_s, s_clocks = time_steps(sstack.step, args.steps, args.warmup, device, ClockSampler(gpu_uuid_id(device)))
+    s_bytes = sstack.bytes_per_step()
+    s_value = aggregate_value(s_bytes, args.steps, world, s_s)
+    decode_inv_s = {"value": s_value, "unit": "GB/s", "ms_per_step": s_s / args.steps * 1e3,
+                    "frac": s_value / world / peaks["hbm_gbs"], "steps": args.steps, "clocks": s_clocks,
+                    "bytes_per_step": s_bytes, "gpu_launches": sstack.launches_per_step * args.steps,
+                    "workload": "the plain decode stack with raw activations: every call is w4a16_gemv_s(x, s), "
+                                "x / s formed inside the kernel (bit-identical x')"}
+    del sstack
+    torch.cuda.empty_cache()
+
     # ---- head 2: prefill GEMM at M=2048, timed over at least 150 ms
     pre = PrefillGemm(device)
     pre.capture()
@@ -704,7 +730,7 @@ def run_gpu(args):
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
             "gemm": gemm, "decode_sweep": sweep, "tiny": tiny, "pack": pack, "crossover": crossover,
-            "decode_prefetch_hint": decode_pf, "decode_fused": decode_fused}
+            "decode_prefetch_hint": decode_pf, "decode_fused": decode_fused, "decode_inv_s_fused": decode_inv_s}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     elif rank == 0:

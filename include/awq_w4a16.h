@@ -170,6 +170,21 @@ awq_status w4a16_gemv(const uint16_t* d_x, const uint32_t* d_qweight, const uint
                       const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
                       void* d_workspace, size_t workspace_bytes, awq_stream_t stream);
 
+/*
+ * w4a16_gemv_s -- w4a16_gemv with the AWQ activation scaling fused in: d_x holds the RAW activations x and
+ * d_s the per-channel AWQ scale s ([K] fp16, device, 16-byte aligned); the kernel uses
+ * x'_mk = fp16_rne(x_mk / s_k), bit-identical to awq_apply_inv_scale (the correctly rounded fp32 quotient
+ * of two fp16 values rounds to the same fp16 as the exact quotient), so y equals
+ * w4a16_gemv(awq_apply_inv_scale(x, s)) bit for bit.  [AWQ/GPTQ] section 2.1 (3) (activations divided
+ * by s at inference); [AutoAWQ] "fused modules" (the separate scaling pass disappears).  x is staged in
+ * shared memory, which bounds M x K per pass: AWQ_ERR_UNSUPPORTED when it does not fit (every M = 1
+ * shape with K <= 32768 fits).  Other arguments, workspace and errors: as w4a16_gemv; d_s NULL gives
+ * AWQ_ERR_INVALID_ARG.
+ */
+awq_status w4a16_gemv_s(const uint16_t* d_x, const uint16_t* d_s, const uint32_t* d_qweight,
+                        const uint16_t* d_scales, const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
+                        void* d_workspace, size_t workspace_bytes, awq_stream_t stream);
+
 /* w4a16_gemm -- prefill path ([AutoAWQ] "GEMM mode", long context): packed tiles staged by the TMA,
  * dequantized to fp16 in shared memory and contracted on the 5th-generation tensor cores (tcgen05,
  * fp32 accumulators in tensor memory). */

@@ -110,3 +110,11 @@ def test_linear_pf_hint_checks(L):
     assert L.w4a16_linear_pf(*args, ctypes.c_void_p(0x10008), 64, None) == 3  # misaligned hint
     assert L.w4a16_linear_pf(*args, F, 24, None) == 1                         # size not a multiple of 16
     assert L.w4a16_linear_pf(F, F, F, F, F, 0, 256, 512, 128, None, 0, F, 64, None) == 1  # M < 1
+
+
+def test_gemv_s_argument_checks(L):
+    F = ctypes.c_void_p(0x10000)
+    assert L.w4a16_gemv_s(F, None, F, F, F, F, 1, 256, 512, 128, None, 0, None) == 1      # s NULL
+    assert L.w4a16_gemv_s(F, ctypes.c_void_p(0x10008), F, F, F, F, 1, 256, 512, 128, None, 0, None) == 3
+    assert L.w4a16_gemv_s(F, F, F, F, F, F, 1, 256, 512, 64, None, 0, None) == 2        # g != 128
+    assert L.w4a16_gemv_s(F, F, F, F, F, F, 0, 256, 512, 128, None, 0, None) == 1       # M < 1

@@ -414,3 +414,41 @@ def test_quantized_linear_within_grid_error_bound():
     S = np.repeat(h2f(sc), 128, axis=1)
     bound = np.abs(h2f(xp)) @ (S * (0.5 + 16 * 2.0**-11)).T
     assert np.all(np.abs(yq - y) <= bound)
+
+
+# ---------------------------------------------------------------- reading used by the fused 1/s GEMV ---
+def _fp16_ties_of_division():
+    """Exact fp16 rounding midpoints x / s = m 2^-25 (m odd, subnormal results) with fp16 x and s."""
+    xs, ss = [], []
+    for k in (3, 5, 7, 11, 13, 99, 1023, 2047):
+        for e in (1, 2, 3, 4):
+            s_ = k * 2.0 ** e
+            for m in range(1, 2048, 2):
+                v = s_ * m * 2.0 ** -25
+                if v < 6.1e-5 and float(np.float16(v)) == v and float(np.float16(s_)) == s_:
+                    xs.append(v)
+                    ss.append(s_)
+    return np.array(xs, np.float16), np.array(ss, np.float16)
+
+
+def test_fp32_quotient_rounds_to_fp16_like_the_oracle_inv_scale():
+    """The fused 1/s GEMV divides in fp32 and rounds once to fp16; oracle_inv_scale divides in fp64.  For
+    fp16 operands the two agree: away from exact midpoints the quotient lies at least 2^-23 (relative) from
+    any fp16 rounding midpoint, more than fp32's half ulp, and an exact midpoint is representable in fp32.
+    Checked here on 400k random operand pairs (all exponents, subnormals, both signs) and on every exact
+    subnormal tie of a family of odd scales (numpy's float32 division and float16 conversion are IEEE)."""
+    rng = np.random.default_rng(5)
+    n = 400000
+    xb = (rng.integers(0, 0x7C00, n).astype(np.uint16) | (rng.integers(0, 2, n).astype(np.uint16) << 15))
+    sb = rng.integers(0x0001, 0x7C00, n).astype(np.uint16)
+    with np.errstate(all="ignore"):
+        q32 = (xb.view(np.float16).astype(np.float32) / sb.view(np.float16).astype(np.float32)).astype(np.float16)
+    ref = O.inv_scale(xb.reshape(1, -1), sb)[0]
+    assert np.array_equal(q32.view(np.uint16), ref)
+    xt, st = _fp16_ties_of_division()
+    assert len(xt) > 500
+    q32 = (xt.astype(np.float32) / st.astype(np.float32)).astype(np.float16).view(np.uint16)
+    ref = O.inv_scale(xt.view(np.uint16).reshape(1, -1), st.view(np.uint16))[0]
+    assert np.array_equal(q32, ref)
+    # the ties really are ties: half of them round down to an even code, half up
+    assert set(np.unique(ref & 1)) == {0}

@@ -25,7 +25,7 @@ __all__ = [
     "AwqError", "PackedWeight", "GROUP", "awq_packed_sizes", "awq_act_scale", "awq_apply_inv_scale", "awq_pack",
     "w4a16_gemv", "w4a16_gemm", "w4a16_linear", "w4a16_gemv_max_m", "w4a16_workspace_bytes",
     "awq_last_device_status", "reserve_workspace", "lib_path", "w4a16_gemv_noalloc",
-    "awq_selftest_wait_timeout", "w4a16_linear_pf",
+    "awq_selftest_wait_timeout", "w4a16_linear_pf", "w4a16_gemv_s",
 ]
 
 
@@ -179,6 +179,26 @@ def w4a16_linear_pf(x, pw: PackedWeight, next_pw: Optional[PackedWeight], out=No
     nxt = (None, 0) if next_pw is None else (next_pw.qweight, next_pw.qweight.numel() * next_pw.qweight.element_size())
     extra = (ctypes.c_void_p(0 if nxt[0] is None else nxt[0].data_ptr()), ctypes.c_size_t(nxt[1]))
     return _linear_call("w4a16_linear_pf", MODE_LINEAR, x, pw, out, workspace, g, extra)
+
+
+def w4a16_gemv_s(x, s, pw: PackedWeight, out=None, workspace=None, g: int = GROUP) -> torch.Tensor:
+    """GEMV on the raw activations x with the AWQ scale s divided out inside the kernel (bit-identical to
+    w4a16_gemv(awq_apply_inv_scale(x, s), pw))."""
+    _need_cuda_fp16(x, "x")
+    _need_cuda_fp16(s, "s")
+    M, K = x.shape
+    if K != pw.K or s.shape != (K,):
+        raise ValueError(f"x has K={K}, s has shape {tuple(s.shape)}, weight has K={pw.K}")
+    N = pw.N
+    if out is not None:
+        _check_out(out, (M, N), x.device)
+    y = torch.empty((M, N), dtype=torch.float16, device=x.device) if out is None else out
+    need = w4a16_workspace_bytes(MODE_GEMV, M, N, K, g)
+    ws = workspace if workspace is not None else (reserve_workspace(need, x.device) if need > 0 else None)
+    st = _lib.load().w4a16_gemv_s(_p(x), _p(s), _p(pw.qweight), _p(pw.scales), _p(pw.qzeros), _p(y), M, N, K, g,
+                                   _p(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream(x.device))
+    _lib.check(st, "w4a16_gemv_s")
+    return y
 
 
 def w4a16_gemv_noalloc(x, pw: PackedWeight, out=None, g: int = GROUP) -> torch.Tensor:

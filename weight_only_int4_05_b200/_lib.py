@@ -14,7 +14,7 @@ EXPORTS = (
     "awq_status_string", "awq_version", "awq_packed_sizes", "awq_act_scale", "awq_apply_inv_scale",
     "awq_pack", "w4a16_gemv", "w4a16_gemm", "w4a16_linear", "w4a16_gemv_max_m", "w4a16_workspace_bytes",
     "awq_last_device_status", "w4a16_gemv_noalloc", "awq_selftest_wait_timeout",
-    "w4a16_linear_pf",
+    "w4a16_linear_pf", "w4a16_gemv_s",
 )
 
 STATUS_NAMES = {0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_UNSUPPORTED", 3: "AWQ_ERR_MISALIGNED",
@@ -61,6 +61,8 @@ def load() -> ctypes.CDLL:
             fn = getattr(lib, name)
             fn.restype = I
             fn.argtypes = [P, P, P, P, P, I, I, I, I, P, Z, P]
+        lib.w4a16_gemv_s.restype = I
+        lib.w4a16_gemv_s.argtypes = [P, P, P, P, P, P, I, I, I, I, P, Z, P]
         lib.w4a16_gemv_noalloc.restype = I
         lib.w4a16_gemv_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, P]
         lib.w4a16_linear_pf.restype = I

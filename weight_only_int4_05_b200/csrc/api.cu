@@ -133,6 +133,19 @@ awq_status w4a16_gemv(const uint16_t* d_x, const uint32_t* d_qweight, const uint
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
+awq_status w4a16_gemv_s(const uint16_t* d_x, const uint16_t* d_s, const uint32_t* d_qweight,
+                        const uint16_t* d_scales, const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g,
+                        void* d_workspace, size_t workspace_bytes, awq_stream_t stream) {
+  awq_status st = check_linear(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g);
+  if (st != AWQ_OK) return st;
+  if (d_s == nullptr) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(d_s) || (d_workspace && !aligned16(d_workspace))) return AWQ_ERR_MISALIGNED;
+  unsigned* status = device_status_ptr();
+  if (status == nullptr) return AWQ_ERR_CUDA;
+  return gemv_launch(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, d_workspace, workspace_bytes, status,
+                     reinterpret_cast<cudaStream_t>(stream), nullptr, 0, d_s);
+}
+
 awq_status w4a16_gemm(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
                       const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g, void* d_workspace,
                       size_t workspace_bytes, awq_stream_t stream) {

@@ -82,6 +82,7 @@ constexpr int kMaxDynSmem = 232448 - 2048;  // opt-in shared memory per block, l
 
 struct GemvParams {
   const uint16_t* x;
+  const uint16_t* s;  // AWQ per-channel scale, divided out of the staged x (DIVS kernels), else NULL
   const uint8_t* qw;
   const uint16_t* scales;
   const uint32_t* qzeros;
@@ -324,7 +325,7 @@ __device__ __forceinline__ void gemv_producer(const GemvParams& p, uint8_t* ring
   }
 }
 
-template <int NT, bool XS>
+template <int NT, bool XS, bool DIVS>
 __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[kSlots];
@@ -402,7 +403,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
   const int rb_l = active ? (wu1 - 1) / G : -1;  // the warp's last row block
 
   bool ok = true;
-  if (XS && active) ok = __all_sync(0xFFFFFFFFu, mbar_wait_backoff(&xbar, 0u, p.status));
+  if (XS && (active || DIVS)) ok = __all_sync(0xFFFFFFFFu, mbar_wait_backoff(&xbar, 0u, p.status));
+  if (DIVS) {
+    // x' = fp16(x / s) in place, every consumer thread taking 8 channels at a time.  The correctly rounded
+    // fp32 quotient rounds to the same fp16 as the exact quotient of two fp16 values (it never lands on an
+    // fp16 rounding midpoint unless the exact quotient is that midpoint), so x' is bit-identical to
+    // awq_apply_inv_scale's fp64 result.
+    if (ok) {
+      const int ct = threadIdx.x;  // 0 .. kNW * 32 - 1
+      for (int m = 0; m < mcount; ++m)
+        for (int k = ct * 8; k < p.K; k += kNW * 32 * 8) {
+          uint4 xv = *reinterpret_cast<const uint4*>(xs + m * p.xpitch + k);
+          const uint4 sv = ldg_cached(p.s + k);
+          uint32_t* xw = reinterpret_cast<uint32_t*>(&xv);
+          const uint32_t* sw = reinterpret_cast<const uint32_t*>(&sv);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const __half2 xh = u32_as_h2(xw[i]), sh = u32_as_h2(sw[i]);
+            const __half lo = __float2half_rn(__fdiv_rn(__low2float(xh), __low2float(sh)));
+            const __half hi = __float2half_rn(__fdiv_rn(__high2float(xh), __high2float(sh)));
+            xw[i] = h2_as_u32(__halves2half2(lo, hi));
+          }
+          *reinterpret_cast<uint4*>(xs + m * p.xpitch + k) = xv;
+        }
+    }
+    named_barrier_sync(3, kNW * 32);  // every consumer sees the divided x'
+  }
   uint4 xb[NT][4];
   if (!XS && active) load_xb<NT>(xrow, g0, t4, xb);
   int rb = rb_f, g = g0;
@@ -492,13 +518,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
 
 namespace {
 
-template <int NT, bool XS>
+template <int NT, bool XS, bool DIVS>
 bool gemv_smem_attr() {
   static bool done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(gemv_kernel<NT, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) !=
+    if (cudaFuncSetAttribute(gemv_kernel<NT, XS, DIVS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) !=
         cudaSuccess)
       return false;
     done[dev] = true;
@@ -519,7 +545,7 @@ struct GemvPlan {
 //  - more row blocks, evenly enough divisible: each CTA takes a balanced run of whole row blocks;
 //  - otherwise (a few row blocks more than CTAs) the units are spread evenly over the CTAs and the row
 //    blocks cut by CTA boundaries are combined in the workspace.
-GemvPlan plan_gemv(int M, int N, int K) {
+GemvPlan plan_gemv(int M, int N, int K, bool divide = false) {
   GemvPlan pl{};
   pl.NT = M <= 8 ? 1 : 2;
   pl.mts = M < 8 * pl.NT ? M : 8 * pl.NT;
@@ -527,7 +553,9 @@ GemvPlan plan_gemv(int M, int N, int K) {
   pl.G = K / 128;
   pl.U = pl.RB * pl.G;
   pl.xpitch = K + kXPad;
-  pl.xs = pl.mts * pl.xpitch * 2 <= kXsMaxBytes &&
+  // x' staged when it fits (the fused 1/s variant divides the staged copy, so it stages whatever fits beside
+  // the rings and partials)
+  pl.xs = (divide || pl.mts * pl.xpitch * 2 <= kXsMaxBytes) &&
           kRingBytes + gemv_xs_bytes(pl.mts, pl.xpitch) + gemv_part_bytes(pl.mts) <= kMaxDynSmem;
   const int p_max = num_sms() * AWQ_GEMV_CTAS_PER_SM;
   pl.S = 1;
@@ -552,29 +580,32 @@ GemvPlan plan_gemv(int M, int N, int K) {
   return pl;
 }
 
-template <int NT, bool XS>
+template <int NT, bool XS, bool DIVS>
 cudaError_t launch_nt(const GemvParams& p, int mcount, cudaStream_t st) {
-  if (!gemv_smem_attr<NT, XS>()) return cudaErrorInvalidValue;
+  if (!gemv_smem_attr<NT, XS, DIVS>()) return cudaErrorInvalidValue;
   const size_t smem = (size_t)kRingBytes + (XS ? gemv_xs_bytes(mcount, p.xpitch) : 0) + gemv_part_bytes(mcount);
-  return launch_pdl(gemv_kernel<NT, XS>, dim3((unsigned)p.P), dim3(kThreads), smem, st, p);
+  return launch_pdl(gemv_kernel<NT, XS, DIVS>, dim3((unsigned)p.P), dim3(kThreads), smem, st, p);
 }
 
 }  // namespace
 
 size_t gemv_workspace_bytes(int M, int N, int K) {
-  const GemvPlan pl = plan_gemv(M, N, K);
+  const GemvPlan pl = plan_gemv(M, N, K);  // the fused 1/s variant has the same plan (same split)
   return pl.part_bytes == 0 ? 0 : kWorkspaceCounterBytes + pl.part_bytes;
 }
 
 awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
                        uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,
-                       cudaStream_t st, const void* pf, size_t pf_bytes) {
-  const GemvPlan pl = plan_gemv(M, N, K);
+                       cudaStream_t st, const void* pf, size_t pf_bytes, const uint16_t* inv_s) {
+  const bool divide = inv_s != nullptr;
+  const GemvPlan pl = plan_gemv(M, N, K, divide);
+  if (divide && !pl.xs) return AWQ_ERR_UNSUPPORTED;  // x / s needs the staged copy
   if ((size_t)pl.RB * 4 > kWorkspaceCounterBytes) return AWQ_ERR_UNSUPPORTED;
   if (pl.part_bytes > 0 && (ws == nullptr || ws_bytes < kWorkspaceCounterBytes + pl.part_bytes))
     return AWQ_ERR_WORKSPACE;
   GemvParams p;
   p.x = x;
+  p.s = inv_s;
   p.qw = reinterpret_cast<const uint8_t*>(qw);
   p.scales = scales;
   p.qzeros = qzeros;
@@ -604,8 +635,9 @@ awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
     p.m0 = m0;
     const int mcount = M - m0 < rows ? M - m0 : rows;
     cudaError_t e;
-    if (pl.NT == 1) e = pl.xs ? launch_nt<1, true>(p, mcount, st) : launch_nt<1, false>(p, mcount, st);
-    else e = pl.xs ? launch_nt<2, true>(p, mcount, st) : launch_nt<2, false>(p, mcount, st);
+    if (divide) e = pl.NT == 1 ? launch_nt<1, true, true>(p, mcount, st) : launch_nt<2, true, true>(p, mcount, st);
+    else if (pl.NT == 1) e = pl.xs ? launch_nt<1, true, false>(p, mcount, st) : launch_nt<1, false, false>(p, mcount, st);
+    else e = pl.xs ? launch_nt<2, true, false>(p, mcount, st) : launch_nt<2, false, false>(p, mcount, st);
     if (e != cudaSuccess) return AWQ_ERR_CUDA;
   }
   return AWQ_OK;

@@ -47,9 +47,12 @@ awq_status pack_launch(const uint16_t* W, const uint16_t* s, int N, int K, uint3
 size_t gemv_workspace_bytes(int M, int N, int K);
 // pf / pf_bytes: optional L2 prefetch of another buffer while the GEMV runs (16-byte aligned, size a
 // multiple of 16; NULL / 0 for none).
+// inv_s: optional AWQ scale; when given, x holds raw activations and the kernel uses x' = fp16(x / s) (the
+// same bits as awq_apply_inv_scale), staged in shared memory (AWQ_ERR_UNSUPPORTED when it does not fit).
 awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
                        uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,
-                       cudaStream_t st, const void* pf = nullptr, size_t pf_bytes = 0);
+                       cudaStream_t st, const void* pf = nullptr, size_t pf_bytes = 0,
+                       const uint16_t* inv_s = nullptr);
 unsigned* device_status_ptr();  // address of the device status word on the current device
 size_t gemm_workspace_bytes(int M, int N, int K);
 awq_status gemm_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
