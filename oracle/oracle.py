@@ -199,3 +199,38 @@ def reference_linear(xp, W, s=None, g: int = GROUP) -> np.ndarray:
     """Whole path from fp16 W: quantize (with s folded) then the fp64 matmul against x'."""
     q, sc, z = quantize(W, s, g)
     return linear_f64(xp, dequant(q, sc, z, g))
+
+
+# ---- fused gate|up with the SiLU activation --------------------------------------------------------
+# "LLM quantization speed-up" (bjdmk.com.cn), "fused modules": several steps of the layer merged into one
+# operation.  Reading: the gated MLP of the Llama-shaped decode workloads, whose gate and up projections
+# read the same x' and meet in silu(gate) * up before the down projection.
+def silu(a) -> np.ndarray:
+    """SiLU, a / (1 + e^-a), in fp64 (e^-a overflowing to inf gives -0 for very negative a)."""
+    a = np.asarray(a, np.float64)
+    with np.errstate(over="ignore"):
+        return a / (1.0 + np.exp(-a))
+
+
+def interleave_gate_up(Wg, Wu) -> np.ndarray:
+    """The [2 NI][K] row order the public header states for awq_pack_gate_up: row 32j + i is gate row
+    16j + i for i < 16 and up row 16j + i - 16 for i >= 16 (NI a multiple of 16)."""
+    Wg = np.asarray(Wg)
+    Wu = np.asarray(Wu)
+    NI, K = Wg.shape
+    assert Wu.shape == (NI, K) and NI % 16 == 0
+    out = np.empty((2 * NI, K), Wg.dtype)
+    blocks = out.reshape(NI // 16, 32, K)
+    blocks[:, :16] = Wg.reshape(NI // 16, 16, K)
+    blocks[:, 16:] = Wu.reshape(NI // 16, 16, K)
+    return out
+
+
+def gate_up_silu_f64(xp, Wqg, Wqu) -> np.ndarray:
+    """h = silu(x' . Wqg^T) * (x' . Wqu^T): both linears in fp64, the product in fp64."""
+    return silu(linear_f64(xp, Wqg)) * linear_f64(xp, Wqu)
+
+
+def gate_up_silu_pairs_f64(xp, qg, scg, zg, qu, scu, zu, ms, js, g: int = GROUP) -> np.ndarray:
+    """h[m, j] for the listed pairs only, from the separately quantized gate and up weights."""
+    return silu(linear_pairs_f64(xp, qg, scg, zg, ms, js, g)) * linear_pairs_f64(xp, qu, scu, zu, ms, js, g)
