@@ -87,6 +87,10 @@ uint16_t oracle_f64_to_f16(double d) {
 /* float -> binary16: widening to double is exact, so this is one rounding of the float's value. */
 uint16_t oracle_f32_to_f16(float f) { return oracle_f64_to_f16((double)f); }
 
+void oracle_f64_to_f16_array(const double* d, size_t n, uint16_t* h) {
+  for (size_t i = 0; i < n; ++i) h[i] = oracle_f64_to_f16(d[i]);
+}
+
 /* ------------------------------------------------------------------------------------------------ */
 /* Step a1: per-channel AWQ scale ([AWQ/GPTQ] 2.1 (2), exponent 0.5).                               */
 void oracle_act_scale(const uint16_t* xcal, int R, int K, uint16_t* s) {
@@ -95,6 +99,17 @@ void oracle_act_scale(const uint16_t* xcal, int R, int K, uint16_t* s) {
     for (int r = 0; r < R; ++r) sum += fabs(oracle_f16_to_f64(xcal[(size_t)r * K + j]));
     double mean = sum / (double)R;
     s[j] = oracle_f64_to_f16(sqrt(mean));
+  }
+}
+
+/* The scale at exponent alpha, for the scale search ([AWQ/GPTQ] 2.1 (3), [LLM-AWQ] "quantization flow"
+ * stage 1): s_j = fp16((mean_r |xcal_rj|)^alpha), mean and power in fp64 (alpha = 0 gives s = 1). */
+void oracle_act_pow(const uint16_t* xcal, int R, int K, double alpha, uint16_t* s) {
+  for (int j = 0; j < K; ++j) {
+    double sum = 0.0;
+    for (int r = 0; r < R; ++r) sum += fabs(oracle_f16_to_f64(xcal[(size_t)r * K + j]));
+    double mean = sum / (double)R;
+    s[j] = oracle_f64_to_f16(alpha == 0.0 ? 1.0 : pow(mean, alpha));
   }
 }
 

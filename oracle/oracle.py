@@ -52,6 +52,8 @@ def _load():
             lib.oracle_f32_to_f16.restype = ctypes.c_uint16
             lib.oracle_f32_to_f16.argtypes = [ctypes.c_float]
             lib.oracle_act_scale.argtypes = [P, I, I, P]
+            lib.oracle_act_pow.argtypes = [P, I, I, ctypes.c_double, P]
+            lib.oracle_f64_to_f16_array.argtypes = [P, ctypes.c_size_t, P]
             lib.oracle_inv_scale.argtypes = [P, P, I, I, P]
             lib.oracle_quantize.argtypes = [P, P, I, I, I, P, P, P]
             lib.oracle_pack.argtypes = [P, P, P, I, I, I, P, P, P]
@@ -60,7 +62,8 @@ def _load():
             lib.oracle_linear_f64.argtypes = [P, P, I, I, I, P]
             lib.oracle_linear_pairs_f64.argtypes = [P, P, P, P, I, I, I, I, P, P, I, P]
             for name in ("oracle_act_scale", "oracle_inv_scale", "oracle_quantize", "oracle_pack",
-                         "oracle_unpack", "oracle_dequant", "oracle_linear_f64", "oracle_linear_pairs_f64"):
+                         "oracle_unpack", "oracle_dequant", "oracle_linear_f64", "oracle_linear_pairs_f64",
+                         "oracle_act_pow", "oracle_f64_to_f16_array"):
                 getattr(lib, name).restype = None
             _lib = lib
     return _lib
@@ -86,6 +89,14 @@ def f16_to_f64(h: int) -> float:
 
 def f64_to_f16(d: float) -> int:
     return int(_load().oracle_f64_to_f16(float(d)))
+
+
+def f64_to_f16_array(d) -> np.ndarray:
+    """Elementwise single-rounding fp64 -> fp16 bits of an array (same shape)."""
+    d = np.ascontiguousarray(d, dtype=np.float64)
+    h = np.empty(d.shape, np.uint16)
+    _load().oracle_f64_to_f16_array(_p(d), d.size, _p(h))
+    return h
 
 
 def f32_to_f16(f: float) -> int:
@@ -234,3 +245,41 @@ def gate_up_silu_f64(xp, Wqg, Wqu) -> np.ndarray:
 def gate_up_silu_pairs_f64(xp, qg, scg, zg, qu, scu, zu, ms, js, g: int = GROUP) -> np.ndarray:
     """h[m, j] for the listed pairs only, from the separately quantized gate and up weights."""
     return silu(linear_pairs_f64(xp, qg, scg, zg, ms, js, g)) * linear_pairs_f64(xp, qu, scu, zu, ms, js, g)
+
+
+# ---- AWQ scale search ----------------------------------------------------------------------------
+# "AWQ and GPTQ algorithms" (jsqmd.com), section 2.1 (3): choose the per-channel scale s that minimises the
+# layer's output error after quantization, ||Q(W diag(s)) (diag(s)^-1 X) - W X||^2 over calibration data X;
+# "LLM-AWQ academic impact" (CSDN mirror), "quantization flow": stage 1 searches, stage 2 quantizes with the
+# result.  Reading: s = (mean |X|)^alpha over a grid alpha = i / n_grid, i = 0 .. n_grid; the quantized layer
+# is the deployed one (x' = fp16(x / s), output rounded to fp16); the error is the squared difference with
+# the exact unquantized x W^T, summed over every calibration row and output.
+def act_pow(xcal, alpha: float) -> np.ndarray:
+    """s_j = fp16((mean_r |xcal_rj|)^alpha), fp64 mean and power; alpha = 0 gives exactly 1."""
+    xcal = _u16(xcal)
+    R, K = xcal.shape
+    s = np.empty(K, np.uint16)
+    _load().oracle_act_pow(_p(xcal), R, K, ctypes.c_double(alpha), _p(s))
+    return s
+
+
+def awq_search_losses(W, xcal, n_grid: int = 20, g: int = GROUP):
+    """Losses L_i, i = 0 .. n_grid, of alpha_i = i / n_grid: L = sum_{r,n} (fp16(y_q) - y)^2 with y = xcal W^T
+    exact and y_q the quantized layer on x' = fp16(xcal / s_i) (every product and sum in fp64)."""
+    W = _u16(W)
+    xcal = _u16(xcal)
+    y = linear_f64(xcal, _u16(W).view(np.float16).astype(np.float32))
+    losses = np.empty(n_grid + 1, np.float64)
+    for i in range(n_grid + 1):
+        s = act_pow(xcal, i / n_grid)
+        yq = linear_f64(inv_scale(xcal, s), dequant(*quantize(W, s, g), g))
+        yq16 = f64_to_f16_array(yq).view(np.float16).astype(np.float64)  # the layer's fp16 output
+        losses[i] = float(np.sum((yq16 - y) ** 2))
+    return losses
+
+
+def awq_search(W, xcal, n_grid: int = 20, g: int = GROUP):
+    """(best index, alpha, s, losses): the first grid point of least loss and its scale."""
+    losses = awq_search_losses(W, xcal, n_grid, g)
+    best = int(np.argmin(losses))
+    return best, best / n_grid, act_pow(xcal, best / n_grid), losses

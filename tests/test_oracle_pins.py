@@ -598,3 +598,78 @@ def test_gate_up_silu_one_hot_closed_form():
     exp_h = np.array([(ai / (1.0 + math.exp(-ai))) * bi for ai, bi in zip(a, b)])
     assert np.max(np.abs(h - exp_h)) < 1e-14
     assert not np.allclose(h, O.silu(b) * a)
+
+
+# ---------------------------------------------------------------- AWQ scale search -----------------
+def test_act_pow_closed_forms():
+    """s(alpha) = fp16(mean|x|^alpha): alpha = 0 gives exactly 1 (even for a zero channel), alpha = 0.5 is
+    the fixed-exponent scale (oracle_act_scale, sqrt), alpha = 1 and 2 on rows of magnitude c give fp16(c)
+    and fp16(c^2)."""
+    rng = np.random.default_rng(41)
+    xcal = f16(rng.standard_normal((16, 256)) * 3)
+    assert np.all(O.act_pow(xcal, 0.0) == 0x3C00)
+    assert np.all(O.act_pow(np.zeros((4, 8), np.uint16), 0.0) == 0x3C00)
+    assert np.array_equal(O.act_pow(xcal, 0.5), O.act_scale(xcal))
+    c = np.array([0.375, 1.5, 3.0, 7.25])
+    rows = np.stack([c, -c, c, -c])  # |x| = c in every row
+    assert np.array_equal(O.act_pow(f16(rows), 1.0), f16(c))
+    assert np.array_equal(O.act_pow(f16(rows), 2.0), f16(c * c))
+
+
+def _rtn_loss_numpy(W, xcal):
+    """Plain RTN layer error with numpy's matmul: the alpha = 0 point of the search, computed on another
+    path (s = 1, so x' = xcal exactly)."""
+    q, sc, z = O.quantize(W, None)
+    Wq = O.dequant(q, sc, z).astype(np.float64)
+    x = h2f(xcal)
+    yq = (x @ Wq.T).astype(np.float16).astype(np.float64)
+    y = x @ h2f(W).T
+    return float(np.sum((yq - y) ** 2))
+
+
+def test_search_alpha_zero_is_plain_rtn():
+    """alpha = 0 reduces the search's loss to the plain round-to-nearest layer (no scaling at all)."""
+    d = synth.linear_inputs(43, 0, 0, 0, 1, 64, 256)
+    W, xcal = d["W"].view(np.uint16), d["xcal"].view(np.uint16)
+    L = O.awq_search_losses(W, xcal, n_grid=4)
+    assert len(L) == 5
+    assert abs(L[0] - _rtn_loss_numpy(W, xcal)) <= 1e-9 * L[0]
+
+
+def test_search_exact_grid_loss_is_output_rounding_only():
+    """Weights exactly on a 4-bit grid (every code 0..15 present in each group) quantize without error at
+    alpha = 0, so the loss there is only the fp16 rounding of the output: sum (fp16(y) - y)^2 (closed form);
+    a loss computed against x' instead of x, or without the square, fails."""
+    rng = np.random.default_rng(47)
+    N, K = 8, 256
+    codes = np.stack([np.concatenate([rng.permutation(np.r_[np.arange(16), rng.integers(0, 16, 112)])
+                                      for _ in range(2)]) for _ in range(N)])
+    S = 2.0 ** rng.integers(-9, -5, (N, 2))
+    z = rng.integers(0, 16, (N, 2))
+    Wd = (codes - np.repeat(z, 128, axis=1)) * np.repeat(S, 128, axis=1)
+    W = f16(Wd)
+    assert np.array_equal(h2f(W), Wd)
+    xcal = f16(rng.standard_normal((8, K)))
+    y = h2f(xcal) @ Wd.T
+    expect = float(np.sum((y.astype(np.float16).astype(np.float64) - y) ** 2))
+    L = O.awq_search_losses(W, xcal, n_grid=2)
+    assert abs(L[0] - expect) <= 1e-12 * max(expect, 1e-30)
+    assert L[1] > L[0]  # any scaling moves the weights off their grid
+
+
+def test_search_protects_a_salient_channel():
+    """Hand-built case in the spirit of the page's importance E[|X_j|] (section 2.1 (2)): channel 0 carries
+    activations 40x larger than the rest while its weights are small, so plain RTN (alpha = 0) wipes them
+    out and the error is dominated by that channel; scaling it up (alpha > 0) must win clearly."""
+    rng = np.random.default_rng(53)
+    N, K, R = 16, 128, 32
+    Wd = 0.02 * rng.standard_normal((N, K))
+    Wd[:, 0] = 0.0015 * rng.standard_normal(N)
+    x = rng.standard_normal((R, K))
+    x[:, 0] *= 40.0
+    best, alpha, s, L = O.awq_search(f16(Wd), f16(x), n_grid=10)
+    assert best > 0 and L[0] > 3.0 * L[best]
+    assert best == int(np.argmin(L)) and alpha == best / 10
+    assert np.array_equal(s, O.act_pow(f16(x), alpha))
+    # the chosen scale is larger on the salient channel than anywhere else
+    assert h2f(s)[0] > h2f(s)[1:].max()
