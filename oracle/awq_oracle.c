@@ -275,3 +275,142 @@ void oracle_linear_pairs_f64(const uint16_t* xp, const uint8_t* q, const uint16_
     out[i] = acc;
   }
 }
+
+/* ------------------------------------------------------------------------------------------------ */
+/* GPTQ ([AWQ/GPTQ] section 3.1: minimise ||W X - W_hat X||_F^2 over the calibration activations, the
+ * Hessian H = X^T X, columns quantized block by block (128 columns) with each column's quantization error
+ * compensated in the columns not yet quantized through the inverse Hessian, the inverse obtained through
+ * Cholesky factorisations, and lazy batch updates of the columns after the block; section 3.3: 1e-6 added
+ * to the diagonal against a singular Hessian).  Everything in fp64 except the grid, which is the same fp32
+ * asymmetric min/max grid as awq_pack (s = 1) applied to the current weights rounded to fp32.              */
+
+/* In-place Cholesky of the symmetric positive definite n x n matrix A (row major): on return the lower
+ * triangle holds L with A = L L^T and the strict upper triangle is zero.  Returns 0, or -1 if A is not
+ * positive definite. */
+int oracle_cholesky_lower(double* A, int n) {
+  for (int j = 0; j < n; ++j) {
+    double d = A[(size_t)j * n + j];
+    for (int k = 0; k < j; ++k) d -= A[(size_t)j * n + k] * A[(size_t)j * n + k];
+    if (!(d > 0.0)) return -1;
+    double ljj = sqrt(d);
+    A[(size_t)j * n + j] = ljj;
+    for (int i = j + 1; i < n; ++i) {
+      double v = A[(size_t)i * n + j];
+      for (int k = 0; k < j; ++k) v -= A[(size_t)i * n + k] * A[(size_t)j * n + k];
+      A[(size_t)i * n + j] = v / ljj;
+    }
+    for (int i = 0; i < j; ++i) A[(size_t)i * n + j] = 0.0;
+  }
+  return 0;
+}
+
+/* U, upper triangular with H^-1 = U^T U: H = L L^T (Cholesky), H^-1 = L^-T L^-1 (L^-1 by forward
+ * substitution), then U = (Cholesky factor of H^-1)^T.  H is n x n row major (not modified). */
+int oracle_gptq_u(const double* H, int n, double* U) {
+  double* L = (double*)malloc(sizeof(double) * (size_t)n * n);
+  double* Li = (double*)calloc((size_t)n * n, sizeof(double));
+  if (!L || !Li) { free(L); free(Li); return -1; }
+  memcpy(L, H, sizeof(double) * (size_t)n * n);
+  int rc = oracle_cholesky_lower(L, n);
+  if (rc == 0) {
+    for (int c = 0; c < n; ++c) /* column c of L^-1: solve L x = e_c */
+      for (int i = c; i < n; ++i) {
+        double v = (i == c) ? 1.0 : 0.0;
+        for (int k = c; k < i; ++k) v -= L[(size_t)i * n + k] * Li[(size_t)k * n + c];
+        Li[(size_t)i * n + c] = v / L[(size_t)i * n + i];
+      }
+    for (int i = 0; i < n; ++i) /* H^-1 = L^-T L^-1 */
+      for (int j = 0; j < n; ++j) {
+        double v = 0.0;
+        for (int k = (i > j ? i : j); k < n; ++k) v += Li[(size_t)k * n + i] * Li[(size_t)k * n + j];
+        U[(size_t)i * n + j] = v;
+      }
+    rc = oracle_cholesky_lower(U, n);
+    if (rc == 0)
+      for (int i = 0; i < n; ++i) /* transpose the lower factor into the upper triangle */
+        for (int j = i + 1; j < n; ++j) {
+          U[(size_t)i * n + j] = U[(size_t)j * n + i];
+          U[(size_t)j * n + i] = 0.0;
+        }
+  }
+  free(L);
+  free(Li);
+  return rc;
+}
+
+/* The grid of one group (the awq_pack grid with s = 1) on the fp32 values v[0 .. g-1]. */
+static void grid_params(const float* v, int g, uint16_t* sch, float* S, int* zi) {
+  float mn = v[0], mx = v[0];
+  for (int e = 1; e < g; ++e) {
+    if (v[e] < mn) mn = v[e];
+    if (v[e] > mx) mx = v[e];
+  }
+  float sc32 = (mx - mn) / 15.0f;
+  if (sc32 < 1e-5f) sc32 = 1e-5f;
+  *sch = oracle_f32_to_f16(sc32);
+  *S = oracle_f16_to_f32(*sch);
+  float zf = rintf(-mn / *S);
+  if (zf < 0.0f) zf = 0.0f;
+  if (zf > 15.0f) zf = 15.0f;
+  *zi = (int)zf;
+}
+
+/* GPTQ of W [N][K] fp16 on calibration rows xcal [R][K] fp16 at group size g; outputs unpacked like
+ * oracle_quantize (q [N][K], sc [N][K/g] fp16, z [N][K/g]).  Returns 0, or -1 if H is not positive
+ * definite. */
+int oracle_gptq(const uint16_t* W, const uint16_t* xcal, int N, int K, int R, int g, double damp, uint8_t* q,
+                uint16_t* sc, uint8_t* z) {
+  const int B = 128, G = K / g;
+  double* H = (double*)calloc((size_t)K * K, sizeof(double));
+  double* U = (double*)malloc(sizeof(double) * (size_t)K * K);
+  double* Wc = (double*)malloc(sizeof(double) * (size_t)N * K);
+  double* E = (double*)malloc(sizeof(double) * (size_t)N * B);
+  float* gv = (float*)malloc(sizeof(float) * (size_t)g);
+  float* S = (float*)malloc(sizeof(float) * (size_t)N);
+  int* zz = (int*)malloc(sizeof(int) * (size_t)N);
+  int rc = -1;
+  if (!H || !U || !Wc || !E || !gv || !S || !zz) goto out;
+  for (int r = 0; r < R; ++r) /* H = X^T X */
+    for (int i = 0; i < K; ++i) {
+      double xi = oracle_f16_to_f64(xcal[(size_t)r * K + i]);
+      if (xi == 0.0) continue;
+      for (int j = 0; j < K; ++j) H[(size_t)i * K + j] += xi * oracle_f16_to_f64(xcal[(size_t)r * K + j]);
+    }
+  for (int i = 0; i < K; ++i) H[(size_t)i * K + i] += damp;
+  if (oracle_gptq_u(H, K, U) != 0) goto out;
+  for (size_t i = 0; i < (size_t)N * K; ++i) Wc[i] = oracle_f16_to_f64(W[i]);
+  for (int b0 = 0; b0 < K; b0 += B) {
+    int b1 = b0 + B < K ? b0 + B : K;
+    for (int i = b0; i < b1; ++i) {
+      if (i % g == 0) { /* a group starts: its grid from the current weights of its g columns */
+        for (int n = 0; n < N; ++n) {
+          for (int e = 0; e < g; ++e) gv[e] = (float)Wc[(size_t)n * K + i + e];
+          grid_params(gv, g, &sc[(size_t)n * G + i / g], &S[n], &zz[n]);
+          z[(size_t)n * G + i / g] = (uint8_t)zz[n];
+        }
+      }
+      double d = U[(size_t)i * K + i];
+      for (int n = 0; n < N; ++n) {
+        double w = Wc[(size_t)n * K + i];
+        float v = rintf((float)w / S[n]) + (float)zz[n];
+        if (v < 0.0f) v = 0.0f;
+        if (v > 15.0f) v = 15.0f;
+        int code = (int)v;
+        q[(size_t)n * K + i] = (uint8_t)code;
+        double err = (w - (double)(code - zz[n]) * (double)S[n]) / d;
+        for (int j = i + 1; j < b1; ++j) Wc[(size_t)n * K + j] -= err * U[(size_t)i * K + j];
+        E[(size_t)n * B + (i - b0)] = err;
+      }
+    }
+    for (int n = 0; n < N; ++n) /* lazy batch update of the columns after the block */
+      for (int j = b1; j < K; ++j) {
+        double v = 0.0;
+        for (int t = 0; t < b1 - b0; ++t) v += E[(size_t)n * B + t] * U[(size_t)(b0 + t) * K + j];
+        Wc[(size_t)n * K + j] -= v;
+      }
+  }
+  rc = 0;
+out:
+  free(H); free(U); free(Wc); free(E); free(gv); free(S); free(zz);
+  return rc;
+}

@@ -53,6 +53,12 @@ def _load():
             lib.oracle_f32_to_f16.argtypes = [ctypes.c_float]
             lib.oracle_act_scale.argtypes = [P, I, I, P]
             lib.oracle_act_pow.argtypes = [P, I, I, ctypes.c_double, P]
+            lib.oracle_cholesky_lower.argtypes = [P, I]
+            lib.oracle_cholesky_lower.restype = I
+            lib.oracle_gptq_u.argtypes = [P, I, P]
+            lib.oracle_gptq_u.restype = I
+            lib.oracle_gptq.argtypes = [P, P, I, I, I, I, ctypes.c_double, P, P, P]
+            lib.oracle_gptq.restype = I
             lib.oracle_f64_to_f16_array.argtypes = [P, ctypes.c_size_t, P]
             lib.oracle_inv_scale.argtypes = [P, P, I, I, P]
             lib.oracle_quantize.argtypes = [P, P, I, I, I, P, P, P]
@@ -283,3 +289,45 @@ def awq_search(W, xcal, n_grid: int = 20, g: int = GROUP):
     losses = awq_search_losses(W, xcal, n_grid, g)
     best = int(np.argmin(losses))
     return best, best / n_grid, act_pow(xcal, best / n_grid), losses
+
+
+
+# ---- GPTQ ----------------------------------------------------------------------------------------
+# "AWQ and GPTQ algorithms" (jsqmd.com), section 3.1: the Hessian H = X^T X of the calibration activations,
+# columns quantized in blocks of 128 with each column's error compensated in the later columns through the
+# inverse Hessian (Cholesky), lazy batch updates after each block; section 3.3: 1e-6 on the diagonal.  The
+# grid is awq_pack's (s = 1), so the result packs into the same layout.
+GPTQ_DAMP = 1e-6
+GPTQ_BLOCK = 128
+
+
+def cholesky_lower(A) -> np.ndarray:
+    A = np.array(A, np.float64, order="C")
+    n = A.shape[0]
+    if _load().oracle_cholesky_lower(_p(A), n) != 0:
+        raise ValueError("not positive definite")
+    return A
+
+
+def gptq_u(H) -> np.ndarray:
+    """Upper triangular U with H^-1 = U^T U."""
+    H = np.ascontiguousarray(H, np.float64)
+    n = H.shape[0]
+    U = np.empty_like(H)
+    if _load().oracle_gptq_u(_p(H), n, _p(U)) != 0:
+        raise ValueError("not positive definite")
+    return U
+
+
+def gptq_quantize(W, xcal, g: int = GROUP, damp: float = GPTQ_DAMP):
+    """GPTQ of W [N][K] on xcal [R][K]: (q [N][K], sc [N][K/g] fp16 bits, z [N][K/g]) like quantize()."""
+    W = _u16(W)
+    xcal = _u16(xcal)
+    N, K = W.shape
+    R = xcal.shape[0]
+    q = np.empty((N, K), np.uint8)
+    sc = np.empty((N, K // g), np.uint16)
+    z = np.empty((N, K // g), np.uint8)
+    if _load().oracle_gptq(_p(W), _p(xcal), N, K, R, g, ctypes.c_double(damp), _p(q), _p(sc), _p(z)) != 0:
+        raise ValueError("the Hessian is not positive definite")
+    return q, sc, z

@@ -673,3 +673,94 @@ def test_search_protects_a_salient_channel():
     assert np.array_equal(s, O.act_pow(f16(x), alpha))
     # the chosen scale is larger on the salient channel than anywhere else
     assert h2f(s)[0] > h2f(s)[1:].max()
+
+
+# ---------------------------------------------------------------- GPTQ ------------------------------
+def _spd(n, seed):
+    rng = np.random.default_rng(seed)
+    A = rng.standard_normal((2 * n, n))
+    return A.T @ A + 0.1 * np.eye(n)
+
+
+def test_cholesky_and_gptq_u_match_numpy():
+    """The oracle's Cholesky and its U (H^-1 = U^T U, upper) against numpy's linalg routines."""
+    H = _spd(48, 61)
+    assert np.allclose(O.cholesky_lower(H), np.linalg.cholesky(H), rtol=0, atol=1e-12)
+    U = O.gptq_u(H)
+    assert np.allclose(U, np.triu(U), atol=0)
+    assert np.allclose(U, np.linalg.cholesky(np.linalg.inv(H)).T, rtol=0, atol=1e-12)
+    assert np.allclose(U.T @ U @ H, np.eye(48), atol=1e-10)
+
+
+@pytest.mark.parametrize("g", [64, 128, 256])
+def test_gptq_identity_hessian_is_rtn(g):
+    """Calibration rows c e_k (R = K): H = c^2 I + 1e-6 I, so U is diagonal and no error reaches another
+    column -- GPTQ must reduce to plain round-to-nearest exactly."""
+    K, N = 256, 40
+    W = synth.linear_inputs(67, 0, 0, 0, 1, N, K)["W"].view(np.uint16)
+    xcal = f16(1.5 * np.eye(K))
+    for a, b in zip(O.gptq_quantize(W, xcal, g), O.quantize(W, None, g)):
+        assert np.array_equal(a, b)
+
+
+def _gptq_slow(W, xcal, g):
+    """GPTQ without blocks or lazy updates: after each column, every later column is corrected at once
+    (numpy fp64 linear algebra; the grid in numpy float32).  Same result as the blocked algorithm up to
+    fp64 rounding."""
+    Wc = h2f(W).copy()
+    N, K = Wc.shape
+    X = h2f(xcal)
+    H = X.T @ X + 1e-6 * np.eye(K)
+    U = np.linalg.cholesky(np.linalg.inv(H)).T
+    q = np.zeros((N, K), np.uint8)
+    sc = np.zeros((N, K // g), np.uint16)
+    z = np.zeros((N, K // g), np.uint8)
+    S = zz = None
+    for i in range(K):
+        if i % g == 0:
+            v = Wc[:, i:i + g].astype(np.float32)
+            mn, mx = v.min(axis=1), v.max(axis=1)
+            s32 = np.maximum((mx - mn) / np.float32(15), np.float32(1e-5))
+            sch = s32.astype(np.float16)
+            S = sch.astype(np.float32)
+            zz = np.clip(np.rint(-mn / S), 0, 15).astype(np.float32)
+            sc[:, i // g] = sch.view(np.uint16)
+            z[:, i // g] = zz.astype(np.uint8)
+        w = Wc[:, i]
+        code = np.clip(np.rint(w.astype(np.float32) / S) + zz, 0, 15)
+        q[:, i] = code.astype(np.uint8)
+        err = (w - (code.astype(np.float64) - zz) * S.astype(np.float64)) / U[i, i]
+        Wc[:, i + 1:] -= np.outer(err, U[i, i + 1:])
+    return q, sc, z
+
+
+@pytest.mark.parametrize("g", [64, 128, 256])
+def test_gptq_blocked_lazy_equals_immediate_updates(g):
+    """The blocked algorithm with lazy batch updates (section 3.1 (3)) equals the column-by-column one
+    written independently above (numpy's inverse and Cholesky, immediate updates of every later column)."""
+    rng = np.random.default_rng(71 + g)
+    N, K, R = 16, 512, 1024
+    W = f16(0.02 * rng.standard_normal((N, K)))
+    mix = np.eye(K) + 0.2 * rng.standard_normal((K, K)) / np.sqrt(K)
+    xcal = f16(rng.standard_normal((R, K)) @ mix)
+    for u, v in zip(O.gptq_quantize(W, xcal, g), _gptq_slow(W, xcal, g)):
+        assert np.array_equal(u, v)
+
+
+@pytest.mark.parametrize("g", [64, 128, 256])
+def test_gptq_lowers_the_layer_error_against_rtn(g):
+    """The objective of section 3.1 (1): on correlated calibration activations GPTQ's output error
+    ||X (W_hat - W)^T||^2 is clearly below plain round-to-nearest's."""
+    rng = np.random.default_rng(79)
+    N, K, R = 64, 256, 512
+    W = f16(0.02 * rng.standard_normal((N, K)))
+    mix = np.eye(K) + 0.3 * rng.standard_normal((K, K)) / 16
+    xcal = f16(rng.standard_normal((R, K)) @ mix)
+    X, Wf = h2f(xcal), h2f(W)
+
+    def loss(q, sc, z):
+        return float(np.sum((X @ (O.dequant(q, sc, z, g).astype(np.float64) - Wf).T) ** 2))
+
+    lg = loss(*O.gptq_quantize(W, xcal, g))
+    lr = loss(*O.quantize(W, None, g))
+    assert lg < 0.85 * lr
