@@ -368,14 +368,17 @@ int oracle_gptq(const uint16_t* W, const uint16_t* xcal, int N, int K, int R, in
   float* gv = (float*)malloc(sizeof(float) * (size_t)g);
   float* S = (float*)malloc(sizeof(float) * (size_t)N);
   int* zz = (int*)malloc(sizeof(int) * (size_t)N);
+  double* gx = (double*)malloc(sizeof(double) * (size_t)K);
   int rc = -1;
-  if (!H || !U || !Wc || !E || !gv || !S || !zz) goto out;
-  for (int r = 0; r < R; ++r) /* H = X^T X */
+  if (!H || !U || !Wc || !E || !gv || !S || !zz || !gx) goto out;
+  for (int r = 0; r < R; ++r) { /* H = X^T X, rows in order */
+    for (int j = 0; j < K; ++j) gx[j] = oracle_f16_to_f64(xcal[(size_t)r * K + j]);
     for (int i = 0; i < K; ++i) {
-      double xi = oracle_f16_to_f64(xcal[(size_t)r * K + i]);
+      double xi = gx[i];
       if (xi == 0.0) continue;
-      for (int j = 0; j < K; ++j) H[(size_t)i * K + j] += xi * oracle_f16_to_f64(xcal[(size_t)r * K + j]);
+      for (int j = 0; j < K; ++j) H[(size_t)i * K + j] += xi * gx[j];
     }
+  }
   for (int i = 0; i < K; ++i) H[(size_t)i * K + i] += damp;
   if (oracle_gptq_u(H, K, U) != 0) goto out;
   for (size_t i = 0; i < (size_t)N * K; ++i) Wc[i] = oracle_f16_to_f64(W[i]);
@@ -411,6 +414,6 @@ int oracle_gptq(const uint16_t* W, const uint16_t* xcal, int N, int K, int R, in
   }
   rc = 0;
 out:
-  free(H); free(U); free(Wc); free(E); free(gv); free(S); free(zz);
+  free(H); free(U); free(Wc); free(E); free(gv); free(S); free(zz); free(gx);
   return rc;
 }
