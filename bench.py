@@ -50,9 +50,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
-def gemv_bytes(M, N, K):
+def gemv_bytes(M, N, K, g=128):
     """Algorithmic bytes of one W4A16 linear: packed weight + scales + zeros, x' and y."""
-    return N * K * BYTES_PER_WEIGHT + 2 * M * K + 2 * M * N
+    return N * K * (0.5 + 2.5 / g) + 2 * M * K + 2 * M * N
 
 
 def pack_bytes(N, K):
@@ -202,13 +202,16 @@ class DecodeStack:
     """32 layers x 7 packed linears, inputs x' and outputs y resident in HBM, one CUDA graph per step."""
 
     def __init__(self, device, seed=0, M=1, layers=LAYERS, inputs_fn=None, prefetch=False, fused=False,
-                 inv_s_fused=False):
+                 inv_s_fused=False, silu=False):
         """inputs_fn(layer, linear, M, N, K) -> (W, xcal, x) fp16 device tensors; default: the seeded
         device generator of the synthetic workload.  prefetch: each call passes the next linear's packed
         weight as an L2 prefetch hint (w4a16_linear_pf).  fused: 4 linears per layer (FUSED_SHAPES).
         inv_s_fused: the resident activations are the raw x and every call is w4a16_gemv_s(x, s), which
-        divides by the AWQ scale inside the kernel (no separate 1/s pass)."""
+        divides by the AWQ scale inside the kernel (no separate 1/s pass).  silu (with fused): the gate|up
+        linear is packed by awq_pack_gate_up and called as w4a16_gate_up_silu, writing silu(gate) * up
+        (14336 columns) instead of both projections."""
         self.prefetch = prefetch
+        self.silu = silu and fused
         self.inv_s_fused = inv_s_fused
         layer_shapes = FUSED_SHAPES if fused else DECODE_SHAPES
         cfg = 6 if fused else 2  # tensor-id namespace of the synthetic inputs
@@ -232,7 +235,11 @@ class DecodeStack:
             else:
                 Wt, xcal, x = inputs_fn(li, j, M, N, K)
             s = W4.awq_act_scale(xcal)
-            pw = W4.awq_pack(Wt, s)
+            gate_up = self.silu and name == "gate_up"
+            if gate_up:  # rows [0, N/2) are the gate projection, [N/2, N) the up projection
+                pw = W4.awq_pack_gate_up(Wt[:N // 2].contiguous(), Wt[N // 2:].contiguous(), s)
+            else:
+                pw = W4.awq_pack(Wt, s)
             xv = self.x_all[xo:xo + M * K].view(M, K)
             if inv_s_fused:
                 xv.copy_(x)
@@ -240,6 +247,8 @@ class DecodeStack:
             else:
                 W4.awq_apply_inv_scale(x, s, out=xv)
             yv = self.y_all[yo:yo + M * N].view(M, N)
+            if gate_up:
+                yv = yv.reshape(-1)[:M * N // 2].view(M, N // 2)
             self.entries.append((pw, xv, yv, K, N))
             xo += M * K
             yo += M * N
@@ -261,6 +270,8 @@ class DecodeStack:
         for i, (pw, xv, yv, _, _) in enumerate(self.entries):
             if self.inv_s_fused:
                 self.W4.w4a16_gemv_s(xv, self.s_list[i], pw, out=yv)
+            elif yv.shape[1] * 2 == pw.N and self.silu:
+                self.W4.w4a16_gate_up_silu(xv, pw, out=yv)
             elif self.prefetch:  # the next linear of the step (the first one of the next step at the end)
                 self.W4.w4a16_linear_pf(xv, pw, self.entries[(i + 1) % n][0], out=yv)
             else:
@@ -284,7 +295,9 @@ class DecodeStack:
 
     def bytes_per_step(self):
         extra = sum(2 * K for _, _, _, K, _ in self.entries) if self.inv_s_fused else 0  # the scale vectors
-        return sum(gemv_bytes(self.M, N, K) for _, _, _, K, N in self.entries) + extra
+        # the gate|up SiLU call writes N / 2 outputs per row instead of N
+        less = sum(self.M * N for pw, _, yv, _, N in self.entries if yv.shape[1] * 2 == N)
+        return sum(gemv_bytes(self.M, N, K) for _, _, _, K, N in self.entries) + extra - less
 
 
 class PrefillGemm:
@@ -571,6 +584,112 @@ def measure_pack(device, peaks, reps):
             "workload": "awq_pack of the 4096 -> 14336 weight, two weights alternating (inputs larger than L2)"}
 
 
+def measure_groups(device, peaks, reps):
+    """Group sizes 64 and 256: the M=1 decode shapes (calls over weight copies larger than L2, one graph) and
+    the M=2048 prefill of the 4096 -> 14336 shape."""
+    import torch
+    import synth
+    import weight_only_int4_05_b200 as W4
+
+    out = []
+    for g in (64, 256):
+        for i, (name, K, N) in enumerate([("q/o", 4096, 4096), ("k/v", 4096, 1024), ("gate/up", 4096, 14336),
+                                          ("down", 14336, 4096)]):
+            Wt, xcal, x = synth.device_linear_inputs(0, synth.tensor_id(1, 0, i, 0), 1, N, K, device)
+            s = W4.awq_act_scale(xcal)
+            xp = W4.awq_apply_inv_scale(x, s)
+            per = N * K * (0.5 + 2.5 / g)
+            pws = [W4.awq_pack(Wt, s, g=g) for _ in range(max(2, int(-(-(512 * 2**20) // per))))]
+            del Wt, xcal, x
+            y = torch.empty((1, N), dtype=torch.float16, device=device)
+            ws = W4.reserve_workspace(max(256, W4.w4a16_workspace_bytes(W4.MODE_GEMV, 1, N, K, g)), device)
+            calls = [(lambda p=pw: W4.w4a16_linear(xp, p, out=y, workspace=ws)) for pw in pws]
+            sec = time_graph_calls(calls, reps, 3, device)
+            gbs = gemv_bytes(1, N, K, g) / sec / 1e9
+            out.append({"g": g, "shape": name, "K": K, "N": N, "M": 1, "us": round(sec * 1e6, 3),
+                        "GB/s": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4)})
+            del pws
+            torch.cuda.empty_cache()
+        K, N, M = 4096, 14336, PREFILL_M
+        Wt, xcal, x = synth.device_linear_inputs(0, synth.tensor_id(3, 0, 0, 0), M, N, K, device)
+        s = W4.awq_act_scale(xcal)
+        xp = W4.awq_apply_inv_scale(x, s)
+        pw = W4.awq_pack(Wt, s, g=g)
+        del Wt, xcal, x
+        y = torch.empty((M, N), dtype=torch.float16, device=device)
+        ws = W4.reserve_workspace(max(256, W4.w4a16_workspace_bytes(W4.MODE_GEMM, M, N, K, g)), device)
+        sec = time_graph_calls([lambda: W4.w4a16_gemm(xp, pw, out=y, workspace=ws)], max(20, reps), 3, device)
+        tf = 2.0 * M * N * K / sec / 1e12
+        out.append({"g": g, "shape": "prefill gate/up", "K": K, "N": N, "M": M, "us": round(sec * 1e6, 2),
+                    "TFLOP/s": round(tf, 1), "frac": round(tf / peaks["bf16_tflops"], 4)})
+        del pw, xp, y
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure_search(device, reps=3):
+    """awq_search_scale on the 4096 -> 4096 projection with 512 calibration rows and 21 grid points, device
+    time per search through the C entry point (preallocated buffers; no host synchronisation inside)."""
+    import ctypes
+    import torch
+    import synth
+    import weight_only_int4_05_b200 as W4
+
+    N, K, R, n_grid = 4096, 4096, 512, 20
+    Wt, xcal, _ = synth.device_linear_inputs(0, synth.tensor_id(8, 0, 0, 0), 1, N, K, device, rows=R)
+    L = W4._lib.load()
+    need = int(L.awq_search_workspace_bytes(N, K, R, 128, n_grid))
+    ws = torch.empty(need, dtype=torch.uint8, device=device)
+    losses = torch.empty(n_grid + 1, dtype=torch.float64, device=device)
+    s = torch.empty(K, dtype=torch.float16, device=device)
+    best = torch.empty(4, dtype=torch.int32, device=device)
+    P = ctypes.c_void_p
+    st = P(torch.cuda.current_stream(device).cuda_stream)
+
+    def run():
+        rc = L.awq_search_scale(P(Wt.data_ptr()), P(xcal.data_ptr()), N, K, R, 128, n_grid, P(losses.data_ptr()),
+                                P(s.data_ptr()), P(best.data_ptr()), P(ws.data_ptr()), need, st)
+        assert rc == 0, rc
+
+    secs, _ = time_steps(run, reps, 1, device)
+    per = secs / reps
+    return {"value": round(per * 1e3, 3), "unit": "ms per search", "N": N, "K": K, "rows": R,
+            "grid_points": n_grid + 1, "ms_per_grid_point": round(per * 1e3 / (n_grid + 1), 3),
+            "best_alpha": int(best[0].item()) / n_grid,
+            "workload": "AWQ scale search of one 4096 -> 4096 linear: per grid point the scale, awq_pack, 1/s, "
+                        "the GEMM over 512 calibration rows and the fp64 squared error"}
+
+
+def measure_gptq(device, reps=2):
+    """gptq_quantize of the 4096 -> 4096 projection on 4096 calibration rows (device time per layer)."""
+    import ctypes
+    import torch
+    import synth
+    import weight_only_int4_05_b200 as W4
+
+    N = K = R = 4096
+    Wt, xcal, _ = synth.device_linear_inputs(0, synth.tensor_id(9, 0, 0, 0), 1, N, K, device, rows=R)
+    L = W4._lib.load()
+    need = int(L.gptq_workspace_bytes(N, K, R, 128))
+    ws = torch.empty(need, dtype=torch.uint8, device=device)
+    out = W4.awq_pack(Wt, None)
+    P = ctypes.c_void_p
+    st = P(torch.cuda.current_stream(device).cuda_stream)
+
+    def run():
+        rc = L.gptq_quantize(P(Wt.data_ptr()), P(xcal.data_ptr()), N, K, R, 128, ctypes.c_double(1e-6),
+                             P(out.qweight.data_ptr()), P(out.scales.data_ptr()), P(out.qzeros.data_ptr()),
+                             P(ws.data_ptr()), need, st)
+        assert rc == 0, rc
+
+    secs, _ = time_steps(run, reps, 1, device)
+    per = secs / reps
+    flops = R * K * K + 2 * K**3 / 3 + N * K * K  # Gram (lower half), Cholesky + inverse, lazy updates (fp64)
+    return {"value": round(per * 1e3, 2), "unit": "ms per layer", "N": N, "K": K, "rows": R,
+            "fp64_GFLOP": round(flops / 1e9, 1), "fp64_TFLOP/s": round(flops / per / 1e12, 2),
+            "workload": "GPTQ of one 4096 -> 4096 linear on 4096 calibration rows into the W4A16 layout"}
+
+
 def measure_crossover(device, reps):
     """Config 4: both modes at every M on the two 70B-class shapes; per M the faster mode and the one
     w4a16_linear picks (calls over weight copies larger than L2, one graph per point)."""
@@ -668,6 +787,20 @@ def run_gpu(args):
     del fstack
     torch.cuda.empty_cache()
 
+    # ---- the fused stack with the gate|up SiLU epilogue (the MLP's activation inside the gate|up call)
+    ustack = DecodeStack(device, fused=True, silu=True)
+    ustack.capture()
+    u_s, u_clocks = time_steps(ustack.step, args.steps, args.warmup, device, ClockSampler(gpu_uuid_id(device)))
+    u_bytes = ustack.bytes_per_step()
+    u_value = aggregate_value(u_bytes, args.steps, world, u_s)
+    decode_fused_silu = {"value": u_value, "unit": "GB/s", "ms_per_step": u_s / args.steps * 1e3,
+                         "frac": u_value / world / peaks["hbm_gbs"], "steps": args.steps, "clocks": u_clocks,
+                         "bytes_per_step": u_bytes, "gpu_launches": ustack.launches_per_step * args.steps,
+                         "workload": "fused decode stack with w4a16_gate_up_silu: 32 layers x {qkv 4096->6144, "
+                                     "o 4096->4096, gate|up+SiLU 4096->2x14336 writing 14336, down 14336->4096}"}
+    del ustack
+    torch.cuda.empty_cache()
+
     # ---- the plain stack with the AWQ 1/s fused into every GEMV (raw x and s in, no separate scaling pass)
     sstack = DecodeStack(device, inv_s_fused=True)
     sstack.capture()
@@ -715,6 +848,9 @@ def run_gpu(args):
     tiny = measure_tiny(device, reps)
     pack = measure_pack(device, peaks, reps)
     crossover = None if args.no_crossover else measure_crossover(device, max(3, reps // 4))
+    groups = measure_groups(device, peaks, reps)
+    search = measure_search(device)
+    gptq = measure_gptq(device)
 
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": seconds / args.steps * 1e3, "higher_is_better": True,
@@ -730,7 +866,8 @@ def run_gpu(args):
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
             "gemm": gemm, "decode_sweep": sweep, "tiny": tiny, "pack": pack, "crossover": crossover,
-            "decode_prefetch_hint": decode_pf, "decode_fused": decode_fused, "decode_inv_s_fused": decode_inv_s}
+            "decode_prefetch_hint": decode_pf, "decode_fused": decode_fused, "decode_inv_s_fused": decode_inv_s,
+            "decode_fused_silu": decode_fused_silu, "group_sizes": groups, "awq_search": search, "gptq": gptq}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     elif rank == 0:
@@ -750,7 +887,8 @@ def run_gpu(args):
 
 def run_profile_case(args):
     """One linear layer launched `warmup + steps` times eagerly on enough weight copies to exceed L2:
-    the small case for detailed ncu captures.  spec = "gemv:K:N:M" or "gemm:K:N:M"."""
+    the small case for detailed ncu captures.  spec = "gemv:K:N:M", "gemm:K:N:M", "silu:K:N:M" (gate|up
+    with the SiLU epilogue, N = 2 NI) or "gptq:K:N:R" (one GPTQ per launch)."""
     import torch
     import synth
     import weight_only_int4_05_b200 as W4
@@ -760,22 +898,33 @@ def run_profile_case(args):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     W4._lib.load()
+    launches = args.warmup + args.steps
+    if mode == "gptq":  # one GPTQ of an N x K weight on M calibration rows per launch
+        Wt, xcal, _ = synth.device_linear_inputs(0, synth.tensor_id(9, 0, 0, 0), 1, N, K, device, rows=M)
+        for _ in range(launches):
+            W4.gptq_quantize(Wt, xcal)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": args.profile_case, "launches": launches,
+                          "device_status": W4.awq_last_device_status()}))
+        return 0
     Wt, xcal, x = synth.device_linear_inputs(0, synth.tensor_id(5, 0, 0, 0), M, N, K, device)
     s = W4.awq_act_scale(xcal)
     xp = W4.awq_apply_inv_scale(x, s)
     copies = max(2, -(-256 * 2**20 // (N * K // 2)))  # > 2 x L2 of packed weights
-    pws = [W4.awq_pack(Wt, s) for _ in range(copies)]
+    if mode == "silu":  # N = NI: the gate and up halves of a 2 NI x K weight
+        pws = [W4.awq_pack_gate_up(Wt[:N // 2].contiguous(), Wt[N // 2:].contiguous(), s) for _ in range(copies)]
+        y = torch.empty((M, N // 2), dtype=torch.float16, device=device)
+    else:
+        pws = [W4.awq_pack(Wt, s) for _ in range(copies)]
+        y = torch.empty((M, N), dtype=torch.float16, device=device)
     del Wt, xcal, x
-    y = torch.empty((M, N), dtype=torch.float16, device=device)
-    fn = {"gemv": W4.w4a16_gemv, "gemm": W4.w4a16_gemm}[mode]
-    for i in range(args.warmup + args.steps):
+    fn = {"gemv": W4.w4a16_gemv, "gemm": W4.w4a16_gemm, "silu": W4.w4a16_gate_up_silu}[mode]
+    for i in range(launches):
         fn(xp, pws[i % copies], out=y)
     torch.cuda.synchronize()
-    print(json.dumps({"profile_case": args.profile_case, "launches": args.warmup + args.steps,
+    print(json.dumps({"profile_case": args.profile_case, "launches": launches,
                       "copies": copies, "device_status": W4.awq_last_device_status()}))
     return 0
-
-
 
 
 def run_crossover(args):

@@ -169,8 +169,9 @@ def linear_inputs(seed: int, config: int, layer: int, linear: int, M: int, N: in
 
 
 # ---- device generator for benchmark-sized stacks (same distributions, torch's CUDA generator) ----
-def device_linear_inputs(seed: int, tid: int, M: int, N: int, K: int, device):
-    """Same distributions as linear_inputs, drawn on `device` with torch.Generator(seed ^ tid)."""
+def device_linear_inputs(seed: int, tid: int, M: int, N: int, K: int, device, rows: int = None):
+    """Same distributions as linear_inputs, drawn on `device` with torch.Generator(seed ^ tid); `rows`
+    calibration rows (default CALIB_ROWS)."""
     import torch
 
     gen = torch.Generator(device=device)
@@ -180,6 +181,6 @@ def device_linear_inputs(seed: int, tid: int, M: int, N: int, K: int, device):
     perm = torch.randperm(K, generator=gen, device=device)
     gain = torch.ones(K, device=device, dtype=torch.float32)
     gain[perm[:n_out]] = OUTLIER_GAIN
-    xcal = (torch.randn((CALIB_ROWS, K), generator=gen, device=device) * gain).half()
+    xcal = (torch.randn((CALIB_ROWS if rows is None else rows, K), generator=gen, device=device) * gain).half()
     x = (torch.randn((M, K), generator=gen, device=device) * gain).half()
     return W, xcal, x

@@ -54,7 +54,11 @@ def test_packed_sizes_match_layout(L, N, K):
 def test_packed_sizes_rejects(L):
     a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
     ref = (ctypes.byref(a), ctypes.byref(b), ctypes.byref(c))
-    assert L.awq_packed_sizes(256, 512, 64, *ref) == 2      # g != 128: unsupported
+    assert L.awq_packed_sizes(256, 512, 32, *ref) == 2      # g not 64 / 128 / 256: unsupported
+    assert L.awq_packed_sizes(256, 512, 96, *ref) == 2
+    assert L.awq_packed_sizes(256, 512, 64, *ref) == 0
+    assert a.value == 256 * 512 // 2 and b.value == 8 * 256 * 2 and c.value == 8 * 256 // 2  # G = 8 at g = 64
+    assert L.awq_packed_sizes(256, 384, 256, *ref) == 1     # K not a multiple of g
     assert L.awq_packed_sizes(0, 512, 128, *ref) == 1
     assert L.awq_packed_sizes(256, 500, 128, *ref) == 1     # K not a multiple of g
     assert L.awq_packed_sizes(256, 512, 128, None, ref[1], ref[2]) == 1
@@ -70,7 +74,8 @@ def _lin(L, fn, M=1, N=256, K=512, g=128, ptrs=(FAKE,) * 5, ws=None, ws_bytes=0)
 
 @pytest.mark.parametrize("fn", ["w4a16_gemv", "w4a16_gemm", "w4a16_linear"])
 def test_linear_argument_checks(L, fn):
-    assert _lin(L, fn, g=64) == 2
+    assert _lin(L, fn, g=32) == 2
+    assert _lin(L, fn, g=256, K=384) == 1  # K % g != 0
     assert _lin(L, fn, M=0) == 1
     assert _lin(L, fn, N=12) == 1          # N % 8 != 0
     assert _lin(L, fn, K=192) == 1         # K % 128 != 0
@@ -82,7 +87,7 @@ def test_linear_argument_checks(L, fn):
 
 def test_pack_and_prep_argument_checks(L):
     P = ctypes.c_void_p
-    assert L.awq_pack(P(FAKE), None, 256, 512, 64, P(FAKE), P(FAKE), P(FAKE), None) == 2
+    assert L.awq_pack(P(FAKE), None, 256, 512, 32, P(FAKE), P(FAKE), P(FAKE), None) == 2
     assert L.awq_pack(P(FAKE), None, 256, 500, 128, P(FAKE), P(FAKE), P(FAKE), None) == 1
     assert L.awq_pack(P(FAKE), None, 0, 512, 128, P(FAKE), P(FAKE), P(FAKE), None) == 1
     assert L.awq_pack(P(FAKE + 8), None, 256, 512, 128, P(FAKE), P(FAKE), P(FAKE), None) == 3
@@ -116,5 +121,47 @@ def test_gemv_s_argument_checks(L):
     F = ctypes.c_void_p(0x10000)
     assert L.w4a16_gemv_s(F, None, F, F, F, F, 1, 256, 512, 128, None, 0, None) == 1      # s NULL
     assert L.w4a16_gemv_s(F, ctypes.c_void_p(0x10008), F, F, F, F, 1, 256, 512, 128, None, 0, None) == 3
-    assert L.w4a16_gemv_s(F, F, F, F, F, F, 1, 256, 512, 64, None, 0, None) == 2        # g != 128
+    assert L.w4a16_gemv_s(F, F, F, F, F, F, 1, 256, 512, 32, None, 0, None) == 2        # g unsupported
     assert L.w4a16_gemv_s(F, F, F, F, F, F, 0, 256, 512, 128, None, 0, None) == 1       # M < 1
+
+
+def test_gate_up_argument_checks(L):
+    P, F = ctypes.c_void_p, ctypes.c_void_p(FAKE)
+    assert L.awq_pack_gate_up(F, F, None, 24, 512, 128, F, F, F, None) == 1      # NI % 16 != 0
+    assert L.awq_pack_gate_up(F, None, None, 32, 512, 128, F, F, F, None) == 1   # NULL up weight
+    assert L.awq_pack_gate_up(F, F, None, 32, 512, 32, F, F, F, None) == 2       # unsupported g
+    assert L.awq_pack_gate_up(P(FAKE + 8), F, None, 32, 512, 128, F, F, F, None) == 3
+    assert L.w4a16_gate_up_silu(F, F, F, F, F, 1, 24, 512, 128, None, 0, None) == 1  # NI % 16 != 0
+    assert L.w4a16_gate_up_silu(F, F, F, F, F, 0, 32, 512, 128, None, 0, None) == 1  # M < 1
+    assert L.w4a16_gate_up_silu(F, F, F, F, F, 1, 32, 512, 32, None, 0, None) == 2   # unsupported g
+    assert L.w4a16_gate_up_silu(F, F, F, F, P(FAKE + 8), 1, 32, 512, 128, None, 0, None) == 3
+
+
+def test_search_argument_checks(L):
+    P, F = ctypes.c_void_p, ctypes.c_void_p(FAKE)
+    args = lambda N=64, K=256, R=8, g=128, n=4: (F, F, N, K, R, g, n, F, F, F, F, 1 << 30, None)  # noqa: E731
+    assert L.awq_search_scale(*args(n=0)) == 1
+    assert L.awq_search_scale(*args(R=0)) == 1
+    assert L.awq_search_scale(*args(N=12)) == 1
+    assert L.awq_search_scale(*args(K=200)) == 1
+    assert L.awq_search_scale(*args(g=32)) == 2
+    assert L.awq_search_workspace_bytes(64, 256, 8, 128, 4) > 64 * 256 // 2
+    assert L.awq_search_workspace_bytes(64, 256, 0, 128, 4) == 2**64 - 1
+    bad = list(args())
+    bad[0] = P(FAKE + 8)
+    assert L.awq_search_scale(*bad) == 3
+
+
+def test_gptq_argument_checks(L):
+    P, F = ctypes.c_void_p, ctypes.c_void_p(FAKE)
+    d = ctypes.c_double(1e-6)
+    assert L.gptq_quantize(F, F, 64, 192, 8, 64, d, F, F, F, F, 1 << 30, None) == 1   # K % 128 != 0
+    assert L.gptq_quantize(F, F, 12, 256, 8, 128, d, F, F, F, F, 1 << 30, None) == 1  # N % 8 != 0
+    assert L.gptq_quantize(F, F, 64, 256, 0, 128, d, F, F, F, F, 1 << 30, None) == 1  # R < 1
+    assert L.gptq_quantize(F, F, 64, 384, 8, 256, d, F, F, F, F, 1 << 30, None) == 1  # K % g != 0
+    assert L.gptq_quantize(F, F, 64, 256, 8, 32, d, F, F, F, F, 1 << 30, None) == 2   # g unsupported
+    assert L.gptq_quantize(F, F, 64, 256, 8, 128, ctypes.c_double(-1.0), F, F, F, F, 1 << 30, None) == 1
+    assert L.gptq_quantize(P(FAKE + 8), F, 64, 256, 8, 128, d, F, F, F, F, 1 << 30, None) == 3
+    assert L.gptq_workspace_bytes(64, 256, 8, 128) >= 2 * 256 * 256 * 8 + 64 * 256 * 8
+    assert L.gptq_workspace_bytes(64, 192, 8, 64) == 2**64 - 1
+    assert L.awq_status_string(7) == b"AWQ_ERR_NUMERIC"

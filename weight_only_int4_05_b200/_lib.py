@@ -14,11 +14,12 @@ EXPORTS = (
     "awq_status_string", "awq_version", "awq_packed_sizes", "awq_act_scale", "awq_apply_inv_scale",
     "awq_pack", "w4a16_gemv", "w4a16_gemm", "w4a16_linear", "w4a16_gemv_max_m", "w4a16_workspace_bytes",
     "awq_last_device_status", "w4a16_gemv_noalloc", "awq_selftest_wait_timeout",
-    "w4a16_linear_pf", "w4a16_gemv_s",
+    "w4a16_linear_pf", "w4a16_gemv_s", "awq_pack_gate_up", "w4a16_gate_up_silu", "awq_search_scale",
+    "awq_search_workspace_bytes", "gptq_quantize", "gptq_workspace_bytes",
 )
 
 STATUS_NAMES = {0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_UNSUPPORTED", 3: "AWQ_ERR_MISALIGNED",
-                4: "AWQ_ERR_CUDA", 5: "AWQ_ERR_DEVICE_TIMEOUT", 6: "AWQ_ERR_WORKSPACE"}
+                4: "AWQ_ERR_CUDA", 5: "AWQ_ERR_DEVICE_TIMEOUT", 6: "AWQ_ERR_WORKSPACE", 7: "AWQ_ERR_NUMERIC"}
 MODE_GEMV, MODE_GEMM, MODE_LINEAR = 1, 2, 3
 
 _lock = threading.Lock()
@@ -57,7 +58,17 @@ def load() -> ctypes.CDLL:
         lib.awq_apply_inv_scale.argtypes = [P, P, I, I, P, P]
         lib.awq_pack.restype = I
         lib.awq_pack.argtypes = [P, P, I, I, I, P, P, P, P]
-        for name in ("w4a16_gemv", "w4a16_gemm", "w4a16_linear"):
+        lib.gptq_quantize.restype = I
+        lib.gptq_quantize.argtypes = [P, P, I, I, I, I, ctypes.c_double, P, P, P, P, Z, P]
+        lib.gptq_workspace_bytes.restype = Z
+        lib.gptq_workspace_bytes.argtypes = [I, I, I, I]
+        lib.awq_search_scale.restype = I
+        lib.awq_search_scale.argtypes = [P, P, I, I, I, I, I, P, P, P, P, Z, P]
+        lib.awq_search_workspace_bytes.restype = Z
+        lib.awq_search_workspace_bytes.argtypes = [I, I, I, I, I]
+        lib.awq_pack_gate_up.restype = I
+        lib.awq_pack_gate_up.argtypes = [P, P, P, I, I, I, P, P, P, P]
+        for name in ("w4a16_gemv", "w4a16_gemm", "w4a16_linear", "w4a16_gate_up_silu"):
             fn = getattr(lib, name)
             fn.restype = I
             fn.argtypes = [P, P, P, P, P, I, I, I, I, P, Z, P]

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_NAME = "libawq_w4a16.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
-SOURCES = ["api.cu", "prep.cu", "pack.cu", "gemv.cu", "gemm.cu", "noalloc.cu", "selftest.cu"]
+SOURCES = ["api.cu", "prep.cu", "pack.cu", "gemv.cu", "gemm.cu", "noalloc.cu", "selftest.cu", "search.cu", "gptq.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

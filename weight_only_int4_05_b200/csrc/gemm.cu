@@ -48,6 +48,8 @@ struct GemmParams {
   const uint32_t* qzeros;
   uint16_t* y;
   unsigned* status;
+  int epi;     // 0: y [M][N]; 1: gate|up, y [M][N/2] = silu(row 32j + i) * row 32j + 16 + i (i < 16)
+  int gshift;  // group of k-block kb: kb >> gshift (group size 64 << gshift)
   float* ws_part;    // split-K partial tiles [tile][split][BT][128] fp32 (splits > 1 only)
   unsigned* ws_cnt;  // per-tile arrival counters (zero between calls)
   int M, N, Np, K, KB, BT, ST, tmem_cols;
@@ -56,7 +58,8 @@ struct GemmParams {
 };
 
 // Producer (lane 0 of warp 0).  Four TMA copies per stage: a 3-D box of the codes of the tile's 4 row
-// blocks (2 chunks of 512 B each), 2-D boxes of their scales (4 x 64 B) and zeros (4 x 16 B), and the
+// blocks (2 chunks of 512 B each), 2-D boxes of their scales (4 x 64 B) and zeros (4 x 16 B) of the group
+// the k-block falls in (a k-block of 64 channels never straddles a group of 64, 128 or 256), and the
 // x' tile in the 128-byte swizzle layout.  Row blocks past the end of the weight come back zero-filled.
 struct GemmMaps {
   CUtensorMap x, codes, scales, zeros;
@@ -68,7 +71,7 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps* maps, const GemmPa
   const unsigned tx = (unsigned)p.BT * 128u + 4096u + 256u + 64u;
   const int rb0 = n0 / 32;
   auto issue_w = [&](int kk, int s) {  // kk: k-block index within this CTA's range
-    const int kb = kb0 + kk, g = kb >> 1;
+    const int kb = kb0 + kk, g = kb >> p.gshift;
     uint8_t* st = smem + (size_t)s * stage_bytes(p.BT);
     mbar_arrive_expect_tx(&full[s], tx);
     tma_load_3d(st + off_pk(p.BT), &maps->codes, 0, kb * 2, rb0, &full[s]);
@@ -118,6 +121,32 @@ __device__ __forceinline__ void gemm_mma(const GemmParams& p, uint8_t* smem, uin
     umma_commit(&empty[s]);
   }
   umma_commit(accf);  // also on abort: lets the CTA wait for in-flight MMAs before freeing TMEM
+}
+
+__device__ __forceinline__ float silu_f32(float a) { return a / (1.0f + expf(-a)); }
+
+// Store 16 output columns (tokens t0 + c0 + i) of weight row n (= n0 + 32 q + lane).  Called by all 32 lanes
+// of a warp with a warp-uniform row block: the gate|up epilogue pairs lane l (< 16, gate row) with lane
+// l + 16 (the matching up row) and writes h[t][16 (n / 32) + l].
+__device__ __forceinline__ void epi_store16(const GemmParams& p, int n, int lane, int tbase, const float (&v)[16]) {
+  if (p.epi) {
+    const int j = n >> 5;  // row block (N is a multiple of 32 for gate|up)
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float up = __shfl_down_sync(0xFFFFFFFFu, v[i], 16);
+      const int t = tbase + i;
+      if (lane < 16 && n < p.N && t < p.M)
+        p.y[(size_t)t * (p.N / 2) + 16 * j + lane] = __half_as_ushort(__float2half_rn(silu_f32(v[i]) * up));
+    }
+    return;
+  }
+  if (n < p.N) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int t = tbase + i;
+      if (t < p.M) p.y[(size_t)t * p.N + n] = __half_as_ushort(__float2half_rn(v[i]));
+    }
+  }
 }
 
 // Dequant role then epilogue; r = 0..127 is the weight row of the tile this thread owns.
@@ -187,13 +216,10 @@ __device__ __forceinline__ void gemm_dequant_epilogue(const GemmParams& p, uint8
       uint32_t v[16];
       tmem_ld_32x32b_x16(tq + (uint32_t)c0, v);
       tmem_wait_ld();
-      if (n < p.N) {
+      float f[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int t = t0 + c0 + i;
-          if (t < p.M) p.y[(size_t)t * p.N + n] = __half_as_ushort(__float2half_rn(__uint_as_float(v[i])));
-        }
-      }
+      for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]);
+      epi_store16(p, n, lane, t0 + c0, f);
     }
     return;
   }
@@ -232,13 +258,7 @@ __device__ __forceinline__ void gemm_dequant_epilogue(const GemmParams& p, uint8
 #pragma unroll
       for (int i = 0; i < 16; ++i) acc[i] += __ldcg(src + (size_t)(c0 + i) * 128 + row);
     }
-    if (n < p.N) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int t = t0 + c0 + i;
-        if (t < p.M) p.y[(size_t)t * p.N + n] = __half_as_ushort(__float2half_rn(acc[i]));
-      }
-    }
+    epi_store16(p, n, lane, t0 + c0, acc);
   }
   if (threadIdx.x == 64) p.ws_cnt[tile] = 0u;
 }
@@ -354,7 +374,7 @@ struct GemmPlan {
 
 // Split K when the output tiles alone cannot occupy the SMs: as many splits as fit in one wave, each
 // with at least 4 k-blocks.
-GemmPlan plan_gemm(int M, int N, int K) {
+GemmPlan plan_gemm(int M, int N, int K) {  // the same plan for every group size
   GemmPlan g{};
   g.BT = pick_bt(M);
   g.n_tiles = ((N + 31) / 32 * 32 + kBN - 1) / kBN;
@@ -371,22 +391,30 @@ GemmPlan plan_gemm(int M, int N, int K) {
   return g;
 }
 
-size_t gemm_workspace_bytes(int M, int N, int K) {
+size_t gemm_workspace_bytes(int M, int N, int K, int gs) {
+  (void)gs;
   const GemmPlan g = plan_gemm(M, N, K);
   return g.part_bytes == 0 ? 0 : kWorkspaceCounterBytes + g.part_bytes;
 }
 
-awq_status gemm_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
-                       uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,
-                       cudaStream_t st) {
+awq_status gemm_launch(const LinearArgs& a) {
   EncodeTiledFn encode = encode_fn();
   if (encode == nullptr) return AWQ_ERR_CUDA;
+  const int M = a.M, N = a.N, K = a.K;
+  void* ws = a.ws;
+  const size_t ws_bytes = a.ws_bytes;
+  const uint16_t* x = a.x;
+  const uint32_t* qw = a.qw;
+  const uint16_t* scales = a.scales;
+  const uint32_t* qzeros = a.qzeros;
   GemmParams p;
   p.qw = reinterpret_cast<const uint4*>(qw);
   p.scales = scales;
   p.qzeros = qzeros;
-  p.y = y;
-  p.status = dev_status;
+  p.y = a.y;
+  p.status = a.status;
+  p.epi = a.epi;
+  p.gshift = a.g == 64 ? 0 : a.g == 128 ? 1 : 2;
   p.M = M;
   p.N = N;
   p.Np = (N + 31) / 32 * 32;
@@ -411,7 +439,7 @@ awq_status gemm_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
 
   GemmMaps maps;
   const cuuint32_t estr[3] = {1, 1, 1};
-  const cuuint64_t RB = (cuuint64_t)p.Np / 32, G = (cuuint64_t)K / 128;
+  const cuuint64_t RB = (cuuint64_t)p.Np / 32, G = (cuuint64_t)K / (cuuint64_t)a.g;
   {  // x' [M][K] fp16, 64 x BT boxes in the 128-byte swizzle layout
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
@@ -449,7 +477,7 @@ awq_status gemm_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
       return AWQ_ERR_CUDA;
   }
   const dim3 grid((unsigned)g.n_tiles, (unsigned)g.t_tiles, (unsigned)g.splits);
-  cudaError_t e = launch_pdl(gemm_kernel, grid, dim3(kGemmThreads), (size_t)smem, st, maps, p);
+  cudaError_t e = launch_pdl(gemm_kernel, grid, dim3(kGemmThreads), (size_t)smem, a.st, maps, p);
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 

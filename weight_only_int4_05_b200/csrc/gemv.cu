@@ -2,20 +2,22 @@
 //
 // y[m][n] = sum_g S[n][g] * sum_{k in g} (q[n][k] - z[n][g]) * x'[m][k]   for up to 8 * NT rows of x' per pass.
 //
-// Units.  The packed layout stores each (32-row block rb, 128-channel group g) as 2048 contiguous bytes of
-// codes, and its 32 scales (64 B) and 32 zero nibbles (16 B) contiguously in the unit-major scale and zero
-// arrays, so unit u = rb * G + g is one stretch of each.  Each of the P CTAs owns a balanced contiguous range
+// Units.  The packed layout stores each (32-row block rb, group g of GS = 64, 128 or 256 channels) as 16 * GS
+// contiguous bytes of codes (GS / 32 tiles of 32 rows x 32 channels), and its 32 scales (64 B) and 32 zero
+// nibbles (16 B) contiguously in the unit-major scale and zero arrays, so unit u = rb * G + g is one stretch
+// of each.  Each of the P CTAs owns a balanced contiguous range
 // of units (q = U / P, one more for the first U % P CTAs); its kNW consumer warps split that range into
 // contiguous sub-ranges, and each consumer warp has its own ring of kRing shared-memory slots.
 //
 // Warp roles.  One producer warp per CTA fills every slot with TMA bulk copies -- the codes, scales and zeros
-// of kSU consecutive units, three copies completing on the slot's "full" mbarrier -- and refills a slot when
+// of the 8 KB of consecutive units a slot holds, three copies completing on the slot's "full" mbarrier -- and
+// refills a slot when
 // its consumer has released it on the slot's "empty" mbarrier.  Slot j of the CTA (warp j / kRing, ring index j % kRing) is
 // served by producer lane j % 32: a thread completes about one bulk copy per ~770 cycles whatever its size,
 // and a copy waiting behind another one stalls its thread, so spreading the slots over the lanes keeps the
 // copies in parallel and keeps every issue stall off the consumer warps.
 //
-// Arithmetic: the tensor cores, fp32 accumulation.  One unit is two 16-row halves x 8 steps of
+// Arithmetic: the tensor cores, fp32 accumulation.  One unit is two 16-row halves x GS / 16 steps of
 // mma.sync m16n8k16 (A = weights, 16 rows x 16 channels; B = x', 16 channels x 8 rows of x'; C = fp32).
 // Lane (g = lane / 4, t = lane % 4) reads word t of rows g and g + 8 of each 32-channel chunk c (conflict-
 // free 4-byte shared loads).  The nibble order of a word makes (w & 0x000F000F) | 0x64006400 the fp16 pair
@@ -25,8 +27,13 @@
 // A fragment for one MMA: its k slots {2t, 2t+1} and {2t+8, 2t+9} stand for channels 32c + 8t + {0, 1}
 // and + {2, 3} (or + {4..7}), and the B fragment holds x' at the same channels, so every product
 // (q - z) * x' is formed exactly in fp32 and summed in fp32.  Each half runs two independent MMA chains
-// (even and odd chunks).  After the 8 steps of a group the fp32 sum of each row is multiplied by the row's
+// (even and odd chunks).  After the steps of a group the fp32 sum of each row is multiplied by the row's
 // scale and added to the row's fp32 output accumulator.  Nothing is summed in fp16.
+//
+// Epilogue.  Plain: y = fp16(sum).  Gate|up (epi = 1, the weight packed by awq_pack_gate_up, rows 0..15 of
+// row block j the gate rows 16j..16j+15 and rows 16..31 the up rows 16j..16j+15): the output has N / 2
+// columns, h[m][16j + i] = fp16(silu(sum of row i) * sum of row 16 + i), silu(a) = a / (1 + e^-a), in fp32
+// on the final sums, so the gate and up products never round to fp16 in between.
 //
 // Before griddepcontrol.wait a kernel touches only its weights: the producer fills the first kRing slots of
 // every consumer before the wait, so with programmatic dependent launch the next kernel's weight stream
@@ -46,19 +53,11 @@
 namespace awq {
 
 // ------------------------------------------------------------------------------------------ constants
-constexpr int kUnitCodeBytes = 2048;
-#ifndef AWQ_GEMV_SLOT_UNITS
-#define AWQ_GEMV_SLOT_UNITS 4
-#endif
-// A ring slot holds kSU consecutive units of a warp's range: their codes (kSU x 2 KB), then their scales
-// (kSU x 64 B), then their zeros (kSU x 16 B) -- three copies per slot, since consecutive units are
-// contiguous in all three arrays.  Few large copies keep the bytes in flight high: a thread gets only about
-// one bulk copy serviced at a time, and under load a copy takes the full memory latency.
-constexpr int kSU = AWQ_GEMV_SLOT_UNITS;
-static_assert((kSU & (kSU - 1)) == 0 && kSU >= 1 && kSU <= 8, "units per slot: 1, 2, 4 or 8");
-constexpr int kSlotScaleOff = kSU * kUnitCodeBytes;
-constexpr int kSlotZeroOff = kSlotScaleOff + kSU * 64;
-constexpr int kSlotStride = (kSU * 2128 + 127) / 128 * 128;
+// A ring slot holds kSlotCodeBytes of codes of consecutive units of a warp's range, then their scales
+// (64 B per unit) and zeros (16 B per unit) -- three copies per slot, since consecutive units are contiguous
+// in all three arrays.  Few large copies keep the bytes in flight high: a thread gets only about one bulk
+// copy serviced at a time, and under load a copy takes the full memory latency.
+constexpr int kSlotCodeBytes = 8192;
 #ifndef AWQ_GEMV_RING
 #define AWQ_GEMV_RING 2
 #endif
@@ -74,8 +73,20 @@ constexpr int kNW = AWQ_GEMV_WARPS;  // consumer warps per CTA (power of two); o
 static_assert((kNW & (kNW - 1)) == 0 && kNW >= 2 && kNW <= 16, "consumer warps per CTA: 2, 4, 8 or 16");
 constexpr int kSlots = kNW * kRing;
 constexpr int kThreads = (kNW + 1) * 32;
-constexpr int kRingBytes = kSlots * kSlotStride;
-static_assert(kRingBytes <= 160 * 1024, "rings too large for shared memory");
+
+// Geometry of a unit and a slot for group size GS.
+template <int GS>
+struct Geo {
+  static_assert(GS == 64 || GS == 128 || GS == 256, "group size 64, 128 or 256");
+  static constexpr int CH = GS / 32;                   // 32-channel chunks (512-B tiles) per unit
+  static constexpr int UB = 16 * GS;                   // code bytes per unit
+  static constexpr int SU = kSlotCodeBytes / UB;       // units per slot: 8, 4, 2
+  static constexpr int SCO = kSlotCodeBytes;           // scales offset in a slot
+  static constexpr int ZO = SCO + SU * 64;             // zeros offset in a slot
+  static constexpr int STRIDE = (ZO + SU * 16 + 127) / 128 * 128;
+  static constexpr int RING = kSlots * STRIDE;         // ring bytes per CTA
+  static_assert(RING <= 160 * 1024, "rings too large for shared memory");
+};
 constexpr int kXsMaxBytes = 36 * 1024;  // x' of one pass staged in shared memory when it fits
 constexpr int kXPad = 32;                // halves of padding per staged row: rows 64 B apart fall in other banks
 constexpr int kMaxDynSmem = 232448 - 2048;  // opt-in shared memory per block, less the static barriers
@@ -87,13 +98,15 @@ struct GemvParams {
   const uint16_t* scales;
   const uint32_t* qzeros;
   uint16_t* y;
+  int epi;  // 0: y[m][n] (ny = N); 1: gate|up SiLU product (ny = N / 2)
+  int ny;   // columns of y
   float* ws_part;
   unsigned* ws_cnt;
   unsigned* status;             // device status word (bounded waits)
   const uint8_t* pf;            // optional: bytes to prefetch into L2 for a later call (NULL: none)
   unsigned long long pf_bytes;  // their size (a multiple of 16)
   unsigned long long pf_share;  // bytes per CTA (a multiple of 16)
-  int U;                        // units = RB * G
+  int U;                        // units = RB * G (G = K / GS)
   int P;                        // CTAs sharing the units: CTA c owns q granules, plus one more if c < r
   int q, r;
   int gran;                     // units per granule: 1, or G when CTA ranges are whole row blocks
@@ -121,26 +134,28 @@ __device__ __forceinline__ void warp_range(int cu0, int n, int w, int& wu0, int&
 // copy (with the barrier's expected byte count) and the scales + zeros copies can come from different lanes,
 // which proceed in parallel; the barrier's phase cannot complete before the arming arrival, so the order in
 // which the lanes' bytes land does not matter.
+template <int GS>
 __device__ __forceinline__ void issue_codes(const GemvParams& p, int u, int c, uint8_t* slot, uint64_t* bar) {
-  mbar_arrive_expect_tx(bar, (unsigned)c * 2128u);
-  bulk_g2s(slot, p.qw + (size_t)u * kUnitCodeBytes, (unsigned)(c * kUnitCodeBytes), bar);
+  mbar_arrive_expect_tx(bar, (unsigned)c * (unsigned)(Geo<GS>::UB + 80));
+  bulk_g2s(slot, p.qw + (size_t)u * Geo<GS>::UB, (unsigned)(c * Geo<GS>::UB), bar);
 }
+template <int GS>
 __device__ __forceinline__ void issue_meta(const GemvParams& p, int u, int c, uint8_t* slot, uint64_t* bar) {
-  bulk_g2s(slot + kSlotScaleOff, p.scales + (size_t)u * 32, (unsigned)(c * 64), bar);
-  bulk_g2s(slot + kSlotZeroOff, p.qzeros + (size_t)u * 4, (unsigned)(c * 16), bar);
+  bulk_g2s(slot + Geo<GS>::SCO, p.scales + (size_t)u * 32, (unsigned)(c * 64), bar);
+  bulk_g2s(slot + Geo<GS>::ZO, p.qzeros + (size_t)u * 4, (unsigned)(c * 16), bar);
 }
 
 // One unit: y rows (g + 8i, i = 0..3) x columns (8 nt + 2t + j) += S_row * sum_k (q - z) x'.
 // codes / scl / zer: 32-bit shared addresses of the unit's codes, scales and zeros; xb[nt][c]: x' row 8 nt + g
-// (clamped to the pass), channels 128 grp + 32c + 8t .. + 7, as 16 bytes.
-template <int NT>
+// (clamped to the pass), channels GS grp + 32c + 8t .. + 7, as 16 bytes; CH = GS / 32 chunks.
+template <int NT, int CH>
 __device__ __forceinline__ void unit_mma(uint32_t codes, uint32_t scl, uint32_t zer, int g, int t,
-                                         const uint4 (&xb)[NT][4], float (&yacc)[NT][4][2]) {
-  uint32_t w[2][2][4];  // [half][row g / g + 8][chunk]
+                                         const uint4 (&xb)[NT][CH], float (&yacc)[NT][4][2]) {
+  uint32_t w[2][2][CH];  // [half][row g / g + 8][chunk]
 #pragma unroll
   for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int cc = 0; cc < CH; ++cc) {
       w[h][0][cc] = ld_shared_u32(codes + 512 * cc + 16 * (16 * h + g) + 4 * t);
       w[h][1][cc] = ld_shared_u32(codes + 512 * cc + 16 * (16 * h + g + 8) + 4 * t);
     }
@@ -166,7 +181,7 @@ __device__ __forceinline__ void unit_mma(uint32_t codes, uint32_t scl, uint32_t 
 #pragma unroll
       for (int pr = 0; pr < 2; ++pr) c[nt][h][pr][0] = c[nt][h][pr][1] = c[nt][h][pr][2] = c[nt][h][pr][3] = 0.f;
 #pragma unroll
-  for (int cc = 0; cc < 4; ++cc)
+  for (int cc = 0; cc < CH; ++cc)
 #pragma unroll
     for (int s = 0; s < 2; ++s)
 #pragma unroll
@@ -192,18 +207,35 @@ __device__ __forceinline__ void unit_mma(uint32_t codes, uint32_t scl, uint32_t 
     }
 }
 
-template <int NT>
-__device__ __forceinline__ void load_xb(const uint16_t* const (&xrow)[NT], int grp, int t, uint4 (&xb)[NT][4]) {
+template <int NT, int GS>
+__device__ __forceinline__ void load_xb(const uint16_t* const (&xrow)[NT], int grp, int t,
+                                        uint4 (&xb)[NT][Geo<GS>::CH]) {
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) xb[nt][cc] = ldg_cached(xrow[nt] + grp * 128 + cc * 32 + t * 8);
+    for (int cc = 0; cc < Geo<GS>::CH; ++cc) xb[nt][cc] = ldg_cached(xrow[nt] + grp * GS + cc * 32 + t * 8);
 }
+
+__device__ __forceinline__ float silu_f32(float a) { return a / (1.0f + expf(-a)); }
 
 // Row block r written directly from a warp's fragments.
 template <int NT>
 __device__ __forceinline__ void store_frag(const GemvParams& p, int r, int g, int t, int mcount,
                                            const float (&yacc)[NT][4][2]) {
+  if (p.epi) {  // rows g + 8i (i = 0, 1) are gate rows, g + 8i + 16 the matching up rows
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int m = 8 * nt + 2 * t + j;
+          if (m < mcount)
+            p.y[(size_t)(p.m0 + m) * p.ny + r * 16 + g + 8 * i] =
+                __half_as_ushort(__float2half_rn(silu_f32(yacc[nt][i][j]) * yacc[nt][i + 2][j]));
+        }
+    return;
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int n = r * 32 + g + 8 * i;
@@ -235,8 +267,18 @@ __device__ __forceinline__ void stash_frag(float* part, int g, int t, int mcount
 
 // lane = row of row block r: y[m][32 r + lane] for m < mcount.  (Fixed-size, fully unrolled arrays keep the
 // values in registers: a dynamically indexed array would live in local memory.)
+// Called by all 32 lanes of a warp (the gate|up epilogue exchanges values between lanes l and l + 16).
 template <int NT>
 __device__ __forceinline__ void store_row(const GemvParams& p, int r, int lane, int mcount, const float (&v)[8 * NT]) {
+  if (p.epi) {
+#pragma unroll
+    for (int m = 0; m < 8 * NT; ++m) {
+      const float up = __shfl_down_sync(0xFFFFFFFFu, v[m], 16);
+      if (lane < 16 && m < mcount)
+        p.y[(size_t)(p.m0 + m) * p.ny + r * 16 + lane] = __half_as_ushort(__float2half_rn(silu_f32(v[m]) * up));
+    }
+    return;
+  }
   const int n = r * 32 + lane;
   if (n >= p.N) return;
 #pragma unroll
@@ -282,13 +324,15 @@ __host__ __device__ constexpr int gemv_xs_bytes(int rows, int xpitch) { return (
 // Producer warp.  Lane L serves CTA slot j = L % kSlotLanes (consumer warp j / kRing, ring index j % kRing):
 // lanes below kSlotLanes issue the slot's codes copy (and arm its barrier), lanes from kSlotLanes on issue its
 // scales and zeros when there are enough lanes, so the big and small copies of a slot are serviced in
-// parallel.  The warp's slot sequence number sq = 0, 1, ... covers its units [sq * kSU, sq * kSU + kSU); ring
-// index si takes the sequence numbers si, si + kRing, ...  The first use of each slot is issued at once
+// parallel.  The warp's slot sequence number sq = 0, 1, ... covers its units [sq * kSU, sq * kSU + kSU) (kSU
+// units per slot); ring index si takes the sequence numbers si, si + kRing, ...  The first use of each slot is issued at once
 // (before any dependency wait), later ones when the consumer has released the slot.
 constexpr int kSlotLanes = kSlots <= 16 ? kSlots : 32;  // lanes that issue codes; kSlots <= 16: one more lane for meta
 static_assert(kSlots <= 32, "one producer warp serves at most 32 slots");
+template <int GS>
 __device__ __forceinline__ void gemv_producer(const GemvParams& p, uint8_t* ring, uint64_t* full, uint64_t* empty,
                                               int cu0, int n, int lane) {
+  constexpr int kSU = Geo<GS>::SU;
   const bool split = kSlots <= 16;
   const int j = split ? lane % 16 : lane;
   const bool does_codes = lane < kSlotLanes, does_meta = split ? (lane >= 16 && j < kSlots) : does_codes;
@@ -296,11 +340,11 @@ __device__ __forceinline__ void gemv_producer(const GemvParams& p, uint8_t* ring
   int wu0, nw;
   warp_range(cu0, n, j / kRing, wu0, nw);
   const int si = j % kRing;
-  uint8_t* slot = ring + (size_t)j * kSlotStride;
+  uint8_t* slot = ring + (size_t)j * Geo<GS>::STRIDE;
   auto issue = [&](int sq) {
     const int u = wu0 + sq * kSU, c = min(kSU, nw - sq * kSU);
-    if (does_codes) issue_codes(p, u, c, slot, &full[j]);
-    if (does_meta) issue_meta(p, u, c, slot, &full[j]);
+    if (does_codes) issue_codes<GS>(p, u, c, slot, &full[j]);
+    if (does_meta) issue_meta<GS>(p, u, c, slot, &full[j]);
   };
   int next = si;  // next slot sequence number to issue
   if (next * kSU < nw) {
@@ -325,8 +369,10 @@ __device__ __forceinline__ void gemv_producer(const GemvParams& p, uint8_t* ring
   }
 }
 
-template <int NT, bool XS, bool DIVS>
+template <int NT, bool XS, bool DIVS, int GS>
 __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
+  using Ge = Geo<GS>;
+  constexpr int kSU = Ge::SU, CH = Ge::CH;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[kSlots];
   __shared__ __align__(8) uint64_t empty[kSlots];
@@ -338,8 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
   const int cu0 = cta_first_unit(p, c), n = cta_units(p, c), cu1 = cu0 + n;
   const int mcount = min(8 * NT, p.M - p.m0);
   uint8_t* ring = smem;
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + kRingBytes);
-  float* s_part = reinterpret_cast<float*>(smem + kRingBytes + (XS ? gemv_xs_bytes(mcount, p.xpitch) : 0));
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + Ge::RING);
+  float* s_part = reinterpret_cast<float*>(smem + Ge::RING + (XS ? gemv_xs_bytes(mcount, p.xpitch) : 0));
 
   for (int j = threadIdx.x; j < kSlots; j += kThreads) {
     mbar_init(&full[j], 1);
@@ -357,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
       for (unsigned long long o = a; o < e; o += 32768ull)
         prefetch_l2_bulk(p.pf + o, (unsigned)(e - o < 32768ull ? e - o : 32768ull));
     }
-    gemv_producer(p, ring, full, empty, cu0, n, lane);
+    gemv_producer<GS>(p, ring, full, empty, cu0, n, lane);
     return;
   }
 
@@ -367,17 +413,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
   warp_range(cu0, n, warp, wu0, nw);
   const int wu1 = wu0 + nw;
   const bool active = nw > 0;
-  const uint32_t ring_addr = smem_u32(ring) + (uint32_t)(warp * kRing * kSlotStride);
+  const uint32_t ring_addr = smem_u32(ring) + (uint32_t)(warp * kRing * Ge::STRIDE);
   const uint32_t empty_addr = smem_u32(&empty[warp * kRing]);
 #if AWQ_GEMV_L2_PREFETCH
   // Before the dependency wait the consumers are idle: each asks for its whole range of codes (32 KB per
   // lane, lanes in parallel) and of scales and zeros to be brought towards L2, so HBM streams at full rate
   // from the kernel's start and the producer's ring copies mostly hit L2.
   if (active) {
-    const int chunks = (nw * kUnitCodeBytes + 32767) / 32768;
+    const int chunks = (nw * Ge::UB + 32767) / 32768;
     for (int ch = lane; ch < chunks; ch += 30) {
       const int off = ch * 32768;
-      prefetch_l2_bulk(p.qw + (size_t)wu0 * kUnitCodeBytes + off, (unsigned)min(32768, nw * kUnitCodeBytes - off));
+      prefetch_l2_bulk(p.qw + (size_t)wu0 * Ge::UB + off, (unsigned)min(32768, nw * Ge::UB - off));
     }
     if (lane == 30) prefetch_l2_bulk(p.scales + (size_t)wu0 * 32, (unsigned)(nw * 64));
     if (lane == 31) prefetch_l2_bulk(p.qzeros + (size_t)wu0 * 4, (unsigned)(nw * 16));
@@ -429,8 +475,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
     }
     named_barrier_sync(3, kNW * 32);  // every consumer sees the divided x'
   }
-  uint4 xb[NT][4];
-  if (!XS && active) load_xb<NT>(xrow, g0, t4, xb);
+  uint4 xb[NT][CH];
+  if (!XS && active) load_xb<NT, GS>(xrow, g0, t4, xb);
   int rb = rb_f, g = g0;
   int t = 0;  // units of this warp consumed so far
   while (t < nw && ok) {  // segments: the units of one row block inside this warp's range
@@ -444,23 +490,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
     for (int i = 0; i < seg; ++i, ++t) {
       const int sq = t / kSU, ui = t & (kSU - 1);  // slot sequence number and unit within the slot
       const int si = sq & (kRing - 1);
-      const uint32_t slot = ring_addr + (uint32_t)(si * kSlotStride);
-      uint4 xcur[NT][4];
+      const uint32_t slot = ring_addr + (uint32_t)(si * Ge::STRIDE);
+      uint4 xcur[NT][CH];
       if (XS) {  // B fragments from the staged x'
-        load_xb<NT>(xrow, g + i, t4, xcur);
+        load_xb<NT, GS>(xrow, g + i, t4, xcur);
       } else {  // loaded one unit ahead from global memory; start the next unit's loads
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) xcur[nt][cc] = xb[nt][cc];
-        if (t + 1 < nw) load_xb<NT>(xrow, (g + i + 1 == G) ? 0 : g + i + 1, t4, xb);
+          for (int cc = 0; cc < CH; ++cc) xcur[nt][cc] = xb[nt][cc];
+        if (t + 1 < nw) load_xb<NT, GS>(xrow, (g + i + 1 == G) ? 0 : g + i + 1, t4, xb);
       }
       if (ui == 0) {  // first unit of the slot: wait for its copies
         ok = __all_sync(0xFFFFFFFFu, mbar_wait_backoff(&full[warp * kRing + si], (unsigned)(sq / kRing) & 1u, p.status));
         if (!ok) break;  // warp-uniform
       }
-      unit_mma<NT>(slot + (uint32_t)(ui * kUnitCodeBytes), slot + (uint32_t)(kSlotScaleOff + ui * 64),
-                   slot + (uint32_t)(kSlotZeroOff + ui * 16), g4, t4, xcur, yacc);
+      unit_mma<NT, CH>(slot + (uint32_t)(ui * Ge::UB), slot + (uint32_t)(Ge::SCO + ui * 64),
+                       slot + (uint32_t)(Ge::ZO + ui * 16), g4, t4, xcur, yacc);
       if (ui == kSU - 1 || t == nw - 1) {  // last unit of the slot: every lane has read it; release it
         __syncwarp();
         if (lane == 0) mbar_arrive_addr(empty_addr + 8u * (uint32_t)si);
@@ -518,18 +564,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
 
 namespace {
 
-template <int NT, bool XS, bool DIVS>
+template <int NT, bool XS, bool DIVS, int GS>
 bool gemv_smem_attr() {
   static bool done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(gemv_kernel<NT, XS, DIVS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(gemv_kernel<NT, XS, DIVS, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMaxDynSmem) != cudaSuccess)
       return false;
     done[dev] = true;
   }
   return true;
+}
+
+int ring_bytes(int gs) {
+  return gs == 64 ? Geo<64>::RING : gs == 128 ? Geo<128>::RING : Geo<256>::RING;
 }
 
 struct GemvPlan {
@@ -545,18 +595,14 @@ struct GemvPlan {
 //  - more row blocks, evenly enough divisible: each CTA takes a balanced run of whole row blocks;
 //  - otherwise (a few row blocks more than CTAs) the units are spread evenly over the CTAs and the row
 //    blocks cut by CTA boundaries are combined in the workspace.
-GemvPlan plan_gemv(int M, int N, int K, bool divide = false) {
+GemvPlan plan_gemv(int M, int N, int K, int gs, bool divide = false) {
   GemvPlan pl{};
   pl.NT = M <= 8 ? 1 : 2;
   pl.mts = M < 8 * pl.NT ? M : 8 * pl.NT;
   pl.RB = (N + 31) / 32;
-  pl.G = K / 128;
+  pl.G = K / gs;
   pl.U = pl.RB * pl.G;
   pl.xpitch = K + kXPad;
-  // x' staged when it fits (the fused 1/s variant divides the staged copy, so it stages whatever fits beside
-  // the rings and partials)
-  pl.xs = (divide || pl.mts * pl.xpitch * 2 <= kXsMaxBytes) &&
-          kRingBytes + gemv_xs_bytes(pl.mts, pl.xpitch) + gemv_part_bytes(pl.mts) <= kMaxDynSmem;
   const int p_max = num_sms() * AWQ_GEMV_CTAS_PER_SM;
   pl.S = 1;
   pl.part_bytes = 0;
@@ -577,53 +623,67 @@ GemvPlan plan_gemv(int M, int N, int K, bool divide = false) {
   }
   pl.q = pl.U / pl.gran / pl.P;
   pl.r = pl.U / pl.gran % pl.P;
+  // x' staged in shared memory when it fits and each warp's range covers at least a third of the groups (a
+  // warp with few units reads only its own groups' x' more cheaply from global memory: measured on the M = 1
+  // decode shapes, q/o 4.83 -> 4.51 us and down 11.08 -> 10.96 us unstaged, gate/up 10.64 vs 10.96 staged).
+  // The fused 1/s variant divides the staged copy, so it stages whatever fits beside the rings and partials.
+  const int units_per_warp = pl.U / pl.P / kNW;
+  pl.xs = (divide || (pl.mts * pl.xpitch * 2 <= kXsMaxBytes && 3 * units_per_warp >= pl.G)) &&
+          ring_bytes(gs) + gemv_xs_bytes(pl.mts, pl.xpitch) + gemv_part_bytes(pl.mts) <= kMaxDynSmem;
   return pl;
 }
 
-template <int NT, bool XS, bool DIVS>
+template <int NT, bool XS, bool DIVS, int GS>
 cudaError_t launch_nt(const GemvParams& p, int mcount, cudaStream_t st) {
-  if (!gemv_smem_attr<NT, XS, DIVS>()) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)kRingBytes + (XS ? gemv_xs_bytes(mcount, p.xpitch) : 0) + gemv_part_bytes(mcount);
-  return launch_pdl(gemv_kernel<NT, XS, DIVS>, dim3((unsigned)p.P), dim3(kThreads), smem, st, p);
+  if (!gemv_smem_attr<NT, XS, DIVS, GS>()) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)Geo<GS>::RING + (XS ? gemv_xs_bytes(mcount, p.xpitch) : 0) + gemv_part_bytes(mcount);
+  return launch_pdl(gemv_kernel<NT, XS, DIVS, GS>, dim3((unsigned)p.P), dim3(kThreads), smem, st, p);
+}
+
+template <int GS>
+cudaError_t launch_gs(const GemvParams& p, int NT, bool xs, bool divide, int mcount, cudaStream_t st) {
+  if (divide) return NT == 1 ? launch_nt<1, true, true, GS>(p, mcount, st) : launch_nt<2, true, true, GS>(p, mcount, st);
+  if (NT == 1) return xs ? launch_nt<1, true, false, GS>(p, mcount, st) : launch_nt<1, false, false, GS>(p, mcount, st);
+  return xs ? launch_nt<2, true, false, GS>(p, mcount, st) : launch_nt<2, false, false, GS>(p, mcount, st);
 }
 
 }  // namespace
 
-size_t gemv_workspace_bytes(int M, int N, int K) {
-  const GemvPlan pl = plan_gemv(M, N, K);  // the fused 1/s variant has the same plan (same split)
+size_t gemv_workspace_bytes(int M, int N, int K, int g) {
+  const GemvPlan pl = plan_gemv(M, N, K, g);  // the fused 1/s variant has the same plan (same split)
   return pl.part_bytes == 0 ? 0 : kWorkspaceCounterBytes + pl.part_bytes;
 }
 
-awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
-                       uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,
-                       cudaStream_t st, const void* pf, size_t pf_bytes, const uint16_t* inv_s) {
-  const bool divide = inv_s != nullptr;
-  const GemvPlan pl = plan_gemv(M, N, K, divide);
+awq_status gemv_launch(const LinearArgs& a) {
+  const bool divide = a.inv_s != nullptr;
+  const GemvPlan pl = plan_gemv(a.M, a.N, a.K, a.g, divide);
   if (divide && !pl.xs) return AWQ_ERR_UNSUPPORTED;  // x / s needs the staged copy
   if ((size_t)pl.RB * 4 > kWorkspaceCounterBytes) return AWQ_ERR_UNSUPPORTED;
-  if (pl.part_bytes > 0 && (ws == nullptr || ws_bytes < kWorkspaceCounterBytes + pl.part_bytes))
+  if (pl.part_bytes > 0 && (a.ws == nullptr || a.ws_bytes < kWorkspaceCounterBytes + pl.part_bytes))
     return AWQ_ERR_WORKSPACE;
   GemvParams p;
-  p.x = x;
-  p.s = inv_s;
-  p.qw = reinterpret_cast<const uint8_t*>(qw);
-  p.scales = scales;
-  p.qzeros = qzeros;
-  p.y = y;
-  p.ws_cnt = static_cast<unsigned*>(ws);
-  p.ws_part = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWorkspaceCounterBytes) : nullptr;
-  p.status = dev_status;
-  p.pf = pf_bytes > 0 ? static_cast<const uint8_t*>(pf) : nullptr;
-  p.pf_bytes = pf_bytes;
-  p.pf_share = ((pf_bytes + (size_t)pl.P - 1) / (size_t)pl.P + 15) / 16 * 16;
+  p.x = a.x;
+  p.s = a.inv_s;
+  p.qw = reinterpret_cast<const uint8_t*>(a.qw);
+  p.scales = a.scales;
+  p.qzeros = a.qzeros;
+  p.y = a.y;
+  p.epi = a.epi;
+  p.ny = a.epi ? a.N / 2 : a.N;
+  p.ws_cnt = static_cast<unsigned*>(a.ws);
+  p.ws_part = a.ws ? reinterpret_cast<float*>(static_cast<char*>(a.ws) + kWorkspaceCounterBytes) : nullptr;
+  p.status = a.status;
+  p.pf = a.pf_bytes > 0 ? static_cast<const uint8_t*>(a.pf) : nullptr;
+  p.pf_bytes = a.pf_bytes;
+  p.pf_share = ((a.pf_bytes + (size_t)pl.P - 1) / (size_t)pl.P + 15) / 16 * 16;
   p.U = pl.U;
   p.P = pl.P;
   p.q = pl.q;
   p.r = pl.r;
   p.gran = pl.gran;
-  p.M = M;
-  p.N = N;
-  p.K = K;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
   p.G = pl.G;
   p.RB = pl.RB;
   p.S = pl.S;
@@ -631,13 +691,15 @@ awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* sc
   p.xpitch = pl.xpitch;
   // passes of 8 * NT rows run one after the other on the stream and share the workspace
   const int rows = 8 * pl.NT;
-  for (int m0 = 0; m0 < M; m0 += rows) {
+  for (int m0 = 0; m0 < a.M; m0 += rows) {
     p.m0 = m0;
-    const int mcount = M - m0 < rows ? M - m0 : rows;
+    const int mcount = a.M - m0 < rows ? a.M - m0 : rows;
     cudaError_t e;
-    if (divide) e = pl.NT == 1 ? launch_nt<1, true, true>(p, mcount, st) : launch_nt<2, true, true>(p, mcount, st);
-    else if (pl.NT == 1) e = pl.xs ? launch_nt<1, true, false>(p, mcount, st) : launch_nt<1, false, false>(p, mcount, st);
-    else e = pl.xs ? launch_nt<2, true, false>(p, mcount, st) : launch_nt<2, false, false>(p, mcount, st);
+    switch (a.g) {
+      case 64: e = launch_gs<64>(p, pl.NT, pl.xs, divide, mcount, a.st); break;
+      case 256: e = launch_gs<256>(p, pl.NT, pl.xs, divide, mcount, a.st); break;
+      default: e = launch_gs<128>(p, pl.NT, pl.xs, divide, mcount, a.st); break;
+    }
     if (e != cudaSuccess) return AWQ_ERR_CUDA;
   }
   return AWQ_OK;

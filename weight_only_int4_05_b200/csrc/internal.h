@@ -42,21 +42,45 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 awq_status prep_act_scale_launch(const uint16_t* xcal, int R, int K, uint16_t* s, cudaStream_t st);
 awq_status prep_inv_scale_launch(const uint16_t* x, const uint16_t* s, int M, int K, uint16_t* xp,
                                  cudaStream_t st);
-awq_status pack_launch(const uint16_t* W, const uint16_t* s, int N, int K, uint32_t* qw, uint16_t* scales,
-                       uint32_t* qz, cudaStream_t st);
-size_t gemv_workspace_bytes(int M, int N, int K);
-// pf / pf_bytes: optional L2 prefetch of another buffer while the GEMV runs (16-byte aligned, size a
-// multiple of 16; NULL / 0 for none).
-// inv_s: optional AWQ scale; when given, x holds raw activations and the kernel uses x' = fp16(x / s) (the
-// same bits as awq_apply_inv_scale), staged in shared memory (AWQ_ERR_UNSUPPORTED when it does not fit).
-awq_status gemv_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
-                       uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,
-                       cudaStream_t st, const void* pf = nullptr, size_t pf_bytes = 0,
-                       const uint16_t* inv_s = nullptr);
+// Pack N rows of K channels at group size g.  W2 == NULL: row n of the packed weight is W[n].  W2 != NULL
+// (gate|up, N = 2 * NI, NI % 16 == 0): row 32j + i of the packed weight is W[16j + i] for i < 16 and
+// W2[16j + i - 16] for i >= 16.
+awq_status pack_launch(const uint16_t* W, const uint16_t* W2, const uint16_t* s, int N, int K, int g, uint32_t* qw,
+                       uint16_t* scales, uint32_t* qz, cudaStream_t st);
+
+// One linear-layer call as the kernels see it.
+struct LinearArgs {
+  const uint16_t* x = nullptr;
+  const uint32_t* qw = nullptr;
+  const uint16_t* scales = nullptr;
+  const uint32_t* qzeros = nullptr;
+  uint16_t* y = nullptr;
+  int M = 0, N = 0, K = 0, g = 128;
+  int epi = 0;  // 0: y [M][N]; 1: gate|up packed by pack_launch with W2, y [M][N/2] = silu(gate) * up
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  unsigned* status = nullptr;
+  cudaStream_t st = nullptr;
+  const void* pf = nullptr;        // GEMV only: optional L2 prefetch of another buffer (16-B aligned, size % 16 == 0)
+  size_t pf_bytes = 0;
+  const uint16_t* inv_s = nullptr;  // GEMV only: x holds raw activations, the kernel uses x' = fp16(x / s) (the
+                                    // same bits as awq_apply_inv_scale); AWQ_ERR_UNSUPPORTED when x does not
+                                    // fit in shared memory
+};
+size_t gemv_workspace_bytes(int M, int N, int K, int g);
+awq_status gemv_launch(const LinearArgs& a);
+size_t gemm_workspace_bytes(int M, int N, int K, int g);
+awq_status gemm_launch(const LinearArgs& a);
 unsigned* device_status_ptr();  // address of the device status word on the current device
-size_t gemm_workspace_bytes(int M, int N, int K);
-awq_status gemm_launch(const uint16_t* x, const uint32_t* qw, const uint16_t* scales, const uint32_t* qzeros,
-                       uint16_t* y, int M, int N, int K, void* ws, size_t ws_bytes, unsigned* dev_status,
+// GPTQ (gptq.cu): workspace bytes and the launch sequence (arguments validated by the caller).
+size_t gptq_workspace_bytes(int N, int K);
+awq_status gptq_launch(const uint16_t* W, const uint16_t* xcal, int N, int K, int R, int g, double damp,
+                       uint32_t* qw, uint16_t* scales, uint32_t* qz, void* ws, size_t ws_bytes, unsigned* status,
                        cudaStream_t st);
+// AWQ scale search (search.cu): workspace bytes and the launch sequence (arguments validated by the caller).
+size_t search_workspace_bytes(int N, int K, int R, int g);
+awq_status search_launch(const uint16_t* W, const uint16_t* xcal, int N, int K, int R, int g, int n_grid,
+                         double* losses, uint16_t* s_out, int* best_out, void* ws, size_t ws_bytes,
+                         unsigned* status, cudaStream_t st);
 
 }  // namespace awq

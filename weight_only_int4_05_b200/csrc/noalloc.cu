@@ -42,7 +42,7 @@ extern "C" awq_status w4a16_gemv_noalloc(const uint16_t* d_x, const uint32_t* d_
   using namespace awq;
   awq_status st = check_linear(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g);
   if (st != AWQ_OK) return st;
-  const size_t need = gemv_workspace_bytes(M, N, K);
+  const size_t need = gemv_workspace_bytes(M, N, K, g);
   if (need > kNoAllocScratchBytes) return AWQ_ERR_WORKSPACE;
   void* scratch = noalloc_scratch_address();
   if (scratch == nullptr) return AWQ_ERR_CUDA;
@@ -52,5 +52,19 @@ extern "C" awq_status w4a16_gemv_noalloc(const uint16_t* d_x, const uint32_t* d_
   // Only a split plan touches the scratch; a plan without split row blocks needs no clearing (and a
   // memset between two GEMVs would keep the second from overlapping the first).
   if (need > 0 && cudaMemsetAsync(scratch, 0, kWorkspaceCounterBytes, s) != cudaSuccess) return AWQ_ERR_CUDA;
-  return gemv_launch(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, scratch, kNoAllocScratchBytes, status, s);
+  LinearArgs a;
+  a.x = d_x;
+  a.qw = d_qweight;
+  a.scales = d_scales;
+  a.qzeros = d_qzeros;
+  a.y = d_y;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.g = g;
+  a.ws = scratch;
+  a.ws_bytes = kNoAllocScratchBytes;
+  a.status = status;
+  a.st = s;
+  return gemv_launch(a);
 }

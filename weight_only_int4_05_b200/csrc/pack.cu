@@ -9,11 +9,15 @@
 //   q = clamp(rint(w'/S) + z, 0, 15).
 //
 // One CTA per run of kPackGroups units of one row block (the units (rb, g0 .. g0+3) are consecutive in all
-// three packed arrays).  Each half-warp takes one (row, group): lane h of the half holds channels 8h..8h+7
+// three packed arrays).  LPG = GS / 8 lanes take one (row, group): lane h of them holds channels 8h..8h+7
 // (one 16-byte load), which are exactly the 8 codes of one packed word, so no lane exchange is needed to
-// assemble it.  Min and max come from four shuffles inside the half-warp.  The units are assembled in shared
-// memory and written with coalesced 16-byte stores.  The kernel streams 2 bytes in and 0.52 bytes out per
-// weight.
+// assemble it.  Min and max come from log2(LPG) shuffles inside those lanes.  The units are assembled in
+// shared memory and written with coalesced 16-byte stores.  The kernel streams 2 bytes in and 0.52 bytes out
+// per weight.
+//
+// Gate|up packing (W2 != NULL): row 32j + i of the packed weight comes from W row 16j + i (i < 16) or W2 row
+// 16j + i - 16 (i >= 16), so the decode and prefill kernels find each gate row and its up row in the same
+// row block, 16 rows apart.
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,33 +28,42 @@ constexpr int kPackGroups = 4;  // units per CTA
 __device__ __forceinline__ float clamp015(float v) { return fminf(fmaxf(v, 0.0f), 15.0f); }
 __device__ __forceinline__ float h2f_bits(uint32_t bits) { return __half2float(__ushort_as_half((unsigned short)bits)); }
 
-__global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W, const __half* __restrict__ s,
-                                                    int N, int K, int G, uint8_t* __restrict__ qw,
-                                                    uint16_t* __restrict__ scales, uint32_t* __restrict__ qz) {
+template <int GS>
+__global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W, const __half* __restrict__ W2,
+                                                    const __half* __restrict__ s, int N, int K, int G,
+                                                    uint8_t* __restrict__ qw, uint16_t* __restrict__ scales,
+                                                    uint32_t* __restrict__ qz) {
   // No griddepcontrol.launch_dependents here: the linear kernels read packed weights before their own
   // dependency wait, so a kernel launched after this one must not start until every packed byte is
   // written.  Without an explicit trigger the dependents start only when this grid has completed.
-  __shared__ __align__(16) uint32_t s_words[kPackGroups * 512];
+  constexpr int LPG = GS / 8;           // lanes per (row, group)
+  constexpr int IPW = 32 / LPG;         // (row, group) items per warp at a time
+  constexpr int NP = 32 / (8 * IPW);    // passes over the 32 rows of the block (8 warps)
+  constexpr int UW = 4 * GS;            // 32-bit code words per unit (16 * GS bytes)
+  __shared__ __align__(16) uint32_t s_words[kPackGroups * UW];
   __shared__ __align__(16) uint16_t s_sc[kPackGroups * 32];
   __shared__ uint8_t s_zb[kPackGroups * 32];
   const int rb = blockIdx.x, g0 = blockIdx.y * kPackGroups;
   const int ng = min(kPackGroups, G - g0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = lane >> 4, hl = lane & 15;
+  const int sub = lane / LPG, hl = lane % LPG;
   pdl_wait_prior_grids();
 
-  // rows 4 * warp + 2 * i + half (i = 0, 1) of the row block; all loads first
-  uint4 raw[2][kPackGroups];
+  // rows (8 * pass + warp) * IPW + sub of the row block; all loads first
+  uint4 raw[NP][kPackGroups];
   uint4 sraw[kPackGroups];
 #pragma unroll
   for (int gi = 0; gi < kPackGroups; ++gi) {
-    const int k0 = (g0 + gi) * 128 + 8 * hl;
+    const int k0 = (g0 + gi) * GS + 8 * hl;
     sraw[gi] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);  // s = 1
     if (gi < ng && s != nullptr) sraw[gi] = *reinterpret_cast<const uint4*>(s + k0);
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int n = rb * 32 + 4 * warp + 2 * i + half;
-      raw[i][gi] = (gi < ng && n < N) ? *reinterpret_cast<const uint4*>(W + (size_t)n * K + k0) : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < NP; ++i) {
+      const int r = (8 * i + warp) * IPW + sub;
+      const int n = rb * 32 + r;
+      const __half* src = W + (size_t)n * K;
+      if (W2 != nullptr) src = (r < 16 ? W : W2) + (size_t)(rb * 16 + (r & 15)) * K;
+      raw[i][gi] = (gi < ng && n < N) ? *reinterpret_cast<const uint4*>(src + k0) : make_uint4(0u, 0u, 0u, 0u);
     }
   }
   // nibble position of channel offset e in a word: even e -> e/2, odd e -> 4 + e/2
@@ -59,8 +72,8 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
     if (gi >= ng) break;  // CTA-uniform
     const uint32_t sw[4] = {sraw[gi].x, sraw[gi].y, sraw[gi].z, sraw[gi].w};
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int r = 4 * warp + 2 * i + half;
+    for (int i = 0; i < NP; ++i) {
+      const int r = (8 * i + warp) * IPW + sub;
       const bool valid = rb * 32 + r < N;
       const uint32_t ww[4] = {raw[i][gi].x, raw[i][gi].y, raw[i][gi].z, raw[i][gi].w};
       float wp[8];
@@ -74,7 +87,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
         mx = fmaxf(mx, wp[e]);
       }
 #pragma unroll
-      for (int off = 8; off > 0; off >>= 1) {  // inside the half-warp
+      for (int off = LPG / 2; off > 0; off >>= 1) {  // inside the LPG lanes of this (row, group)
         mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
         mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
       }
@@ -89,7 +102,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
         word |= code << (4 * ((e & 1) ? 4 + (e >> 1) : (e >> 1)));
       }
       // word hl & 3 of row r in the unit's chunk hl >> 2 (chunk = 512 B = 128 words, row = 4 words)
-      s_words[gi * 512 + (hl >> 2) * 128 + r * 4 + (hl & 3)] = valid ? word : 0u;
+      s_words[gi * UW + (hl >> 2) * 128 + r * 4 + (hl & 3)] = valid ? word : 0u;
       if (hl == 0) {
         s_sc[gi * 32 + r] = valid ? __half_as_ushort(sch) : (uint16_t)0;
         s_zb[gi * 32 + r] = valid ? (uint8_t)(int)zf : (uint8_t)0;
@@ -98,8 +111,8 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
   }
   __syncthreads();
   const size_t u0 = (size_t)rb * G + g0;  // first unit of this CTA; its ng units are consecutive
-  uint4* dst = reinterpret_cast<uint4*>(qw + u0 * 2048);
-  for (int idx = threadIdx.x; idx < ng * 128; idx += 256) dst[idx] = reinterpret_cast<const uint4*>(s_words)[idx];
+  uint4* dst = reinterpret_cast<uint4*>(qw + u0 * (size_t)(16 * GS));
+  for (int idx = threadIdx.x; idx < ng * UW / 4; idx += 256) dst[idx] = reinterpret_cast<const uint4*>(s_words)[idx];
   if (threadIdx.x < ng * 4) {
     reinterpret_cast<uint4*>(scales + u0 * 32)[threadIdx.x] = reinterpret_cast<const uint4*>(s_sc)[threadIdx.x];
     uint32_t zw = 0u;
@@ -110,13 +123,21 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
   __threadfence();  // the packed units are performed at device scope before this CTA exits
 }
 
-awq_status pack_launch(const uint16_t* W, const uint16_t* s, int N, int K, uint32_t* qw, uint16_t* scales,
-                       uint32_t* qz, cudaStream_t st) {
+awq_status pack_launch(const uint16_t* W, const uint16_t* W2, const uint16_t* s, int N, int K, int g, uint32_t* qw,
+                       uint16_t* scales, uint32_t* qz, cudaStream_t st) {
   const int RB = (N + 31) / 32;
-  const int G = K / 128;
+  const int G = K / g;
   const dim3 grid((unsigned)RB, (unsigned)((G + kPackGroups - 1) / kPackGroups));  // x: row blocks (no 65535 cap)
-  cudaError_t e = launch_pdl(pack_kernel, grid, dim3(256), 0, st, reinterpret_cast<const __half*>(W),
-                             reinterpret_cast<const __half*>(s), N, K, G, reinterpret_cast<uint8_t*>(qw), scales, qz);
+  const __half* w = reinterpret_cast<const __half*>(W);
+  const __half* w2 = reinterpret_cast<const __half*>(W2);
+  const __half* sh = reinterpret_cast<const __half*>(s);
+  uint8_t* q = reinterpret_cast<uint8_t*>(qw);
+  cudaError_t e;
+  switch (g) {
+    case 64: e = launch_pdl(pack_kernel<64>, grid, dim3(256), 0, st, w, w2, sh, N, K, G, q, scales, qz); break;
+    case 256: e = launch_pdl(pack_kernel<256>, grid, dim3(256), 0, st, w, w2, sh, N, K, G, q, scales, qz); break;
+    default: e = launch_pdl(pack_kernel<128>, grid, dim3(256), 0, st, w, w2, sh, N, K, G, q, scales, qz); break;
+  }
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
