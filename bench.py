@@ -753,7 +753,8 @@ def run_gpu(args):
     launches = stack.launches_per_step
     roofline = {"bound": "hbm", "achieved": per_gpu, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": per_gpu / peaks["hbm_gbs"], "traffic": profiled_traffic("gemv_kernel"),
-                "kernel": "gemv_kernel<1, true>", "peak_source": peak_src + " (HBM copy, burst)",
+                "kernel": "gemv_kernel<1, XS, false, 128> (x' staged for gate/up, read directly for the others)",
+                "peak_source": peak_src + " (HBM copy, burst)",
                 "bytes_per_launch": bytes_step / launches, "launch_us": seconds / args.steps / launches * 1e6}
 
     # ---- e2e through the public API with host buffers
