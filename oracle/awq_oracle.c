@@ -123,11 +123,13 @@ void oracle_inv_scale(const uint16_t* x, const uint16_t* s, int M, int K, uint16
 }
 
 /* ------------------------------------------------------------------------------------------------ */
-/* Steps a2-a5: fold s into W and quantize each (row, group) with the asymmetric 4-bit grid.
- *   W [N][K] fp16, s [K] fp16 or NULL (= 1).  Outputs, unpacked: q [N][K] codes 0..15,
- *   sc [N][K/g] fp16 scales, z [N][K/g] zeros 0..15.                                                 */
-void oracle_quantize(const uint16_t* W, const uint16_t* s, int N, int K, int g, uint8_t* q, uint16_t* sc,
-                     uint8_t* z) {
+/* Steps a2-a5: fold s into W and quantize each (row, group) with the asymmetric grid of w_bit bits,
+ * qmax = 2^w_bit - 1 (15 for the pages' 4 bits; 7 for the 3-bit grid):
+ *   W [N][K] fp16, s [K] fp16 or NULL (= 1).  Outputs, unpacked: q [N][K] codes 0..qmax,
+ *   sc [N][K/g] fp16 scales, z [N][K/g] zeros 0..qmax.                                               */
+void oracle_quantize_bits(const uint16_t* W, const uint16_t* s, int N, int K, int g, int w_bit, uint8_t* q,
+                          uint16_t* sc, uint8_t* z) {
+  const float qmax = (float)((1 << w_bit) - 1);
   int G = K / g;
   float* wp = (float*)malloc(sizeof(float) * (size_t)g);
   for (int n = 0; n < N; ++n) {
@@ -147,13 +149,13 @@ void oracle_quantize(const uint16_t* W, const uint16_t* s, int N, int K, int g, 
       }
       /* a4: scale (fp16) and zero point */
       float range = mx - mn;
-      float sc32 = range / 15.0f;
+      float sc32 = range / qmax;
       if (sc32 < 1e-5f) sc32 = 1e-5f;
       uint16_t sch = oracle_f32_to_f16(sc32);
       float S = oracle_f16_to_f32(sch);
       float zf = rintf(-mn / S);
       if (zf < 0.0f) zf = 0.0f;
-      if (zf > 15.0f) zf = 15.0f;
+      if (zf > qmax) zf = qmax;
       int zi = (int)zf;
       sc[(size_t)n * G + gi] = sch;
       z[(size_t)n * G + gi] = (uint8_t)zi;
@@ -162,12 +164,17 @@ void oracle_quantize(const uint16_t* W, const uint16_t* s, int N, int K, int g, 
         float r = rintf(wp[e] / S);
         float v = r + (float)zi;
         if (v < 0.0f) v = 0.0f;
-        if (v > 15.0f) v = 15.0f;
+        if (v > qmax) v = qmax;
         q[(size_t)n * K + gi * g + e] = (uint8_t)(int)v;
       }
     }
   }
   free(wp);
+}
+
+void oracle_quantize(const uint16_t* W, const uint16_t* s, int N, int K, int g, uint8_t* q, uint16_t* sc,
+                     uint8_t* z) {
+  oracle_quantize_bits(W, s, N, K, g, 4, q, sc, z);
 }
 
 /* ------------------------------------------------------------------------------------------------ */

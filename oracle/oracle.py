@@ -62,6 +62,7 @@ def _load():
             lib.oracle_f64_to_f16_array.argtypes = [P, ctypes.c_size_t, P]
             lib.oracle_inv_scale.argtypes = [P, P, I, I, P]
             lib.oracle_quantize.argtypes = [P, P, I, I, I, P, P, P]
+            lib.oracle_quantize_bits.argtypes = [P, P, I, I, I, I, P, P, P]
             lib.oracle_pack.argtypes = [P, P, P, I, I, I, P, P, P]
             lib.oracle_unpack.argtypes = [P, P, P, I, I, I, P, P, P]
             lib.oracle_dequant.argtypes = [P, P, P, I, I, I, P]
@@ -69,7 +70,7 @@ def _load():
             lib.oracle_linear_pairs_f64.argtypes = [P, P, P, P, I, I, I, I, P, P, I, P]
             for name in ("oracle_act_scale", "oracle_inv_scale", "oracle_quantize", "oracle_pack",
                          "oracle_unpack", "oracle_dequant", "oracle_linear_f64", "oracle_linear_pairs_f64",
-                         "oracle_act_pow", "oracle_f64_to_f16_array"):
+                         "oracle_act_pow", "oracle_f64_to_f16_array", "oracle_quantize_bits"):
                 getattr(lib, name).restype = None
             _lib = lib
     return _lib
@@ -131,8 +132,8 @@ def inv_scale(x, s) -> np.ndarray:
 
 
 # ---- a2..a5: fold + grid + codes ------------------------------------------------------------------
-def quantize(W, s=None, g: int = GROUP):
-    """Returns (q [N][K] uint8, sc [N][G] uint16 fp16 bits, z [N][G] uint8)."""
+def quantize(W, s=None, g: int = GROUP, w_bit: int = 4):
+    """Returns (q [N][K] uint8, sc [N][G] uint16 fp16 bits, z [N][G] uint8); codes 0 .. 2^w_bit - 1."""
     W = _u16(W)
     N, K = W.shape
     G = K // g
@@ -140,7 +141,7 @@ def quantize(W, s=None, g: int = GROUP):
     sc = np.empty((N, G), np.uint16)
     z = np.empty((N, G), np.uint8)
     sp = None if s is None else _p(_u16(s))
-    _load().oracle_quantize(_p(W), sp, N, K, g, _p(q), _p(sc), _p(z))
+    _load().oracle_quantize_bits(_p(W), sp, N, K, g, w_bit, _p(q), _p(sc), _p(z))
     return q, sc, z
 
 
@@ -173,9 +174,9 @@ def unpack(qw, scales, qz, N: int, K: int, g: int = GROUP):
     return q, sc, z
 
 
-def awq_pack(W, s=None, g: int = GROUP):
+def awq_pack(W, s=None, g: int = GROUP, w_bit: int = 4):
     """Stage-2 "real quantization": fold s, quantize and pack.  Returns (qweight, scales, qzeros)."""
-    return pack(*quantize(W, s, g), g)
+    return pack(*quantize(W, s, g, w_bit), g)
 
 
 # ---- dequant and matmul ---------------------------------------------------------------------------

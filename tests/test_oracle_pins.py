@@ -764,3 +764,36 @@ def test_gptq_lowers_the_layer_error_against_rtn(g):
     lg = loss(*O.gptq_quantize(W, xcal, g))
     lr = loss(*O.quantize(W, None, g))
     assert lg < 0.85 * lr
+
+
+# ---------------------------------------------------------------- 3-bit grid -----------------------
+# "LLM-AWQ academic impact", recommendations: choose 4-bit or 3-bit quantization by the hardware; "10 INT4
+# models on 20 tasks", introduction: AWQ's INT3 results.  The 3-bit grid is the same asymmetric min/max grid
+# with qmax = 7 (codes 0..7), stored in the 4-bit layout.
+@pytest.mark.parametrize("S0,z0", [(0.0078125, 3), (0.5, 7), (0.000244140625, 0)])
+def test_quantize_3bit_reproduces_its_own_grid(S0, z0):
+    rng = np.random.default_rng(int(S0 * 1e6) + z0)
+    codes = np.concatenate([np.arange(8), rng.integers(0, 8, 120)])
+    rng.shuffle(codes)
+    w = (codes.astype(np.float64) - z0) * S0
+    q, sc, z = O.quantize(f16(w[None, :]), None, 128, 3)
+    assert h2f(sc)[0, 0] == S0 and z[0, 0] == z0 and np.array_equal(q[0], codes)
+
+
+def test_quantize_3bit_clamps_and_bound():
+    """All-positive group: z clamps to 0 and the top code to 7; codes never exceed 7; the round-trip bound
+    |w' - (q - z) S| <= S (1/2 + 8 * 2^-11) where no clamp applies; the 3-bit error exceeds the 4-bit one."""
+    w = np.linspace(1.0, 2.0, 128)
+    q, sc, z = O.quantize(f16(w[None, :]), None, 128, 3)
+    assert z[0, 0] == 0 and q.max() == 7
+    W, s = _synthetic_group_rows()
+    q3, sc3, z3 = O.quantize(W, s, 128, 3)
+    assert q3.max() <= 7 and z3.max() <= 7
+    wp = h2f(W) * h2f(s)[None, :]
+    deq3 = O.dequant(q3, sc3, z3).astype(np.float64)
+    S = np.repeat(h2f(sc3), 128, axis=1)
+    assert np.all(np.abs(wp - deq3) <= S * (0.5 + 8 * 2.0**-11))
+    deq4 = O.dequant(*O.quantize(W, s)).astype(np.float64)
+    assert np.mean((deq3 - wp) ** 2) > 3.0 * np.mean((deq4 - wp) ** 2)
+    for a, b in zip(O.quantize(W, s, 128, 4), O.quantize(W, s)):
+        assert np.array_equal(a, b)  # w_bit = 4 is the default grid
