@@ -152,6 +152,17 @@ awq_status awq_pack(const uint16_t* d_W, const uint16_t* d_s, int N, int K, int 
                     uint16_t* d_scales, uint32_t* d_qzeros, awq_stream_t stream);
 
 /*
+ * awq_pack_bits -- awq_pack with the bit width of the grid as a parameter: w_bit = 4 is awq_pack; w_bit = 3 is
+ * the 3-bit grid ([LLM-AWQ] "choose 4-bit or 3-bit quantization by hardware resources"; [INT4-VLM] introduction:
+ * AWQ at INT3): the same asymmetric grid with qmax = 7 (sc32 = max((mx - mn)/7, 1e-5), z and q clamped to
+ * 0..7).  The codes are stored in the same 4-bit layout, so every linear entry point runs the result unchanged;
+ * the 3-bit grid gives its accuracy, not a smaller weight (0.52 bytes per weight as at 4 bits).
+ * Errors: as awq_pack; AWQ_ERR_UNSUPPORTED for w_bit other than 3 or 4.
+ */
+awq_status awq_pack_bits(const uint16_t* d_W, const uint16_t* d_s, int N, int K, int g, int w_bit, uint32_t* d_qweight,
+                         uint16_t* d_scales, uint32_t* d_qzeros, awq_stream_t stream);
+
+/*
  * awq_pack_gate_up -- packs the gate and up projections of a gated MLP (both [NI][K], the same input x)
  * as ONE packed weight of N = 2 * NI rows for w4a16_gate_up_silu ([AutoAWQ] "fused modules": one weight
  * stream and one read of x for both projections).  Row 32j + i of the packed weight is gate row 16j + i

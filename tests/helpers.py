@@ -17,15 +17,15 @@ RELL2_TOL = 2e-3
 class OracleCase:
     """Inputs of one linear layer and everything the oracle derives from them (lazily)."""
 
-    def __init__(self, seed, config, layer, linear, M, N, K, g=O.GROUP):
-        self.M, self.N, self.K, self.g = M, N, K, g
+    def __init__(self, seed, config, layer, linear, M, N, K, g=O.GROUP, w_bit=4):
+        self.M, self.N, self.K, self.g, self.w_bit = M, N, K, g, w_bit
         d = synth.linear_inputs(seed, config, layer, linear, M, N, K)
         self.W = d["W"].view(np.uint16)
         self.xcal = d["xcal"].view(np.uint16)
         self.x = d["x"].view(np.uint16)
         self.s = O.act_scale(self.xcal)
         self.xp = O.inv_scale(self.x, self.s)
-        self.q, self.sc, self.z = O.quantize(self.W, self.s, g)
+        self.q, self.sc, self.z = O.quantize(self.W, self.s, g, w_bit)
         self._packed = None
 
     @property

@@ -165,3 +165,11 @@ def test_gptq_argument_checks(L):
     assert L.gptq_workspace_bytes(64, 256, 8, 128) >= 2 * 256 * 256 * 8 + 64 * 256 * 8
     assert L.gptq_workspace_bytes(64, 192, 8, 64) == 2**64 - 1
     assert L.awq_status_string(7) == b"AWQ_ERR_NUMERIC"
+
+
+def test_pack_bits_argument_checks(L):
+    P, F = ctypes.c_void_p, ctypes.c_void_p(FAKE)
+    assert L.awq_pack_bits(F, None, 256, 512, 128, 5, F, F, F, None) == 2   # w_bit unsupported
+    assert L.awq_pack_bits(F, None, 256, 512, 128, 2, F, F, F, None) == 2
+    assert L.awq_pack_bits(F, None, 256, 500, 128, 3, F, F, F, None) == 1   # K % g != 0
+    assert L.awq_pack_bits(P(FAKE + 8), None, 256, 512, 128, 3, F, F, F, None) == 3

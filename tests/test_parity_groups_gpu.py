@@ -1,7 +1,7 @@
 """GPU parity at group sizes 64 and 256 (the pages' --q_group_size parameter; 128 is covered everywhere
-else): pack bit-exact against the oracle, GEMV (plain and with the 1/s fused), GEMM and the mode choice
-within the linear layer's tolerance, every output at small sizes and sampled outputs at a full decode
-shape."""
+else) and on the 3-bit grid (codes 0..7 in the 4-bit layout): pack bit-exact against the oracle, GEMV (plain
+and with the 1/s fused), GEMM and the mode choice within the linear layer's tolerance, every output at small
+sizes and sampled outputs at a full decode shape."""
 import numpy as np
 import pytest
 import torch
@@ -27,7 +27,7 @@ def host_u32(t):
 def prep(case):
     s = W4.awq_act_scale(dev(case.xcal))
     xp = W4.awq_apply_inv_scale(dev(case.x), s)
-    pw = W4.awq_pack(dev(case.W), s, g=case.g)
+    pw = W4.awq_pack(dev(case.W), s, g=case.g, w_bit=case.w_bit)
     torch.cuda.synchronize()
     qw, sc, qz = case.packed
     assert np.array_equal(host_u32(pw.qweight), qw), "qweight"
@@ -76,3 +76,19 @@ def test_group_size_is_checked():
         W4.w4a16_gemv(xp, pw, g=128)  # the weight was packed with g = 64
     with pytest.raises(W4.AwqError):
         W4.awq_pack(dev(case.W), None, g=32)
+
+
+@pytest.mark.parametrize("g", [64, 128, 256])
+@pytest.mark.parametrize("N,K,M", [(264, 1024, 1), (256, 512, 40), (4096, 4096, 1)])
+def test_3bit_grid_pack_and_linears(g, N, K, M):
+    """awq_pack_bits with w_bit = 3: bit-exact codes 0..7, and both linear modes on them."""
+    case = OracleCase(7, 1, g, 3, M, N, K, g=g, w_bit=3)
+    s, xp, pw = prep(case)
+    assert case.q.max() <= 7
+    ms, ns = sample_pairs(M, N, 2000, seed=g + M)
+    y_ref = case.y_pairs(ms, ns)
+    for name, fn in (("gemv", W4.w4a16_gemv), ("gemm", W4.w4a16_gemm)):
+        y = fn(xp, pw)
+        torch.cuda.synchronize()
+        assert_within_tolerance(y.float().cpu().numpy()[ms, ns], y_ref, f"3-bit {name} g={g} N={N} K={K} M={M}")
+    assert W4.awq_last_device_status() == 0

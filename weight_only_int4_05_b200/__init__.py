@@ -107,8 +107,9 @@ def awq_apply_inv_scale(x: torch.Tensor, s: torch.Tensor, out: Optional[torch.Te
 
 
 def awq_pack(W: torch.Tensor, s: Optional[torch.Tensor] = None, g: int = GROUP,
-             out: Optional[PackedWeight] = None) -> PackedWeight:
-    """Packs W (with s folded in); `out` reuses the three buffers of an earlier PackedWeight of the same shape."""
+             out: Optional[PackedWeight] = None, w_bit: int = 4) -> PackedWeight:
+    """Packs W (with s folded in); `out` reuses the three buffers of an earlier PackedWeight of the same shape.
+    w_bit = 3 quantizes on the 3-bit grid (codes 0..7) in the same 4-bit layout."""
     _need_cuda_fp16(W, "W")
     N, K = W.shape
     if s is not None:
@@ -118,7 +119,11 @@ def awq_pack(W: torch.Tensor, s: Optional[torch.Tensor] = None, g: int = GROUP,
     dev = W.device
     qw, sc, qz = _packed_buffers(N, K, g, dev, out)
     L = _lib.load()
-    _lib.check(L.awq_pack(_p(W), _p(s), N, K, g, _p(qw), _p(sc), _p(qz), _stream(dev)), "awq_pack")
+    if w_bit == 4:
+        _lib.check(L.awq_pack(_p(W), _p(s), N, K, g, _p(qw), _p(sc), _p(qz), _stream(dev)), "awq_pack")
+    else:
+        _lib.check(L.awq_pack_bits(_p(W), _p(s), N, K, g, w_bit, _p(qw), _p(sc), _p(qz), _stream(dev)),
+                   "awq_pack_bits")
     return PackedWeight(qw, sc, qz, N, K, g)
 
 

@@ -112,6 +112,19 @@ awq_status awq_pack(const uint16_t* d_W, const uint16_t* d_s, int N, int K, int 
   return pack_launch(d_W, nullptr, d_s, N, K, g, d_qweight, d_scales, d_qzeros, reinterpret_cast<cudaStream_t>(stream));
 }
 
+awq_status awq_pack_bits(const uint16_t* d_W, const uint16_t* d_s, int N, int K, int g, int w_bit, uint32_t* d_qweight,
+                         uint16_t* d_scales, uint32_t* d_qzeros, awq_stream_t stream) {
+  if (w_bit != 3 && w_bit != 4) return AWQ_ERR_UNSUPPORTED;
+  if (!group_supported(g)) return AWQ_ERR_UNSUPPORTED;
+  if (N < 1 || K < g || K % g != 0 || N > kMaxN || K > kMaxK) return AWQ_ERR_INVALID_ARG;
+  if (!d_W || !d_qweight || !d_scales || !d_qzeros) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(d_W) || (d_s && !aligned16(d_s)) || !aligned16(d_qweight) || !aligned16(d_scales) ||
+      !aligned16(d_qzeros))
+    return AWQ_ERR_MISALIGNED;
+  return pack_launch(d_W, nullptr, d_s, N, K, g, d_qweight, d_scales, d_qzeros, reinterpret_cast<cudaStream_t>(stream),
+                     w_bit);
+}
+
 awq_status awq_pack_gate_up(const uint16_t* d_Wgate, const uint16_t* d_Wup, const uint16_t* d_s, int NI, int K, int g,
                             uint32_t* d_qweight, uint16_t* d_scales, uint32_t* d_qzeros, awq_stream_t stream) {
   if (!group_supported(g)) return AWQ_ERR_UNSUPPORTED;

@@ -12,7 +12,8 @@
 //                       element sums its products over the rows in row order (each product is exact).
 //   chol_panel_kernel,  blocked right-looking Cholesky Hr = L L^T (64 x 64 tiles): each step factors the
 //   chol_update_kernel  diagonal tile, solves the panel below it, and updates the trailing lower triangle.
-//   trtri_row_kernel    Xi = L^-1, one block row per launch (forward substitution over tiles).
+//   trtri_solve_kernel, Xi = L^-1, right-looking: solve one block row (the diagonal tile's forward substitution),
+//   trtri_update_kernel then add its contribution to every later block row at once.
 //   Then U = J Xi J (J the index reversal) is upper triangular with H^-1 = U^T U -- the factor GPTQ's
 //   error compensation uses -- without a second factorisation.
 //   gptq_block_kernel   one 128-column block: a CTA per 32-row block quantizes the columns in order, spreads
@@ -164,44 +165,22 @@ __global__ void __launch_bounds__(256) chol_update_kernel(double* __restrict__ A
     for (int v = 0; v < 4; ++v) A[(size_t)(ti * kT + ty + 16 * u) * K + tj * kT + tx + 16 * v] -= acc[u][v];
 }
 
-// Block row b of Xi = L^-1 (L lower, the factored Hr): CTA c (0 .. b) computes
-//   Xi[b][c] = L[b][b]^-1 (delta_bc I - sum_{k = c}^{b-1} L[b][k] Xi[k][c]).
-__global__ void __launch_bounds__(256) trtri_row_kernel(const double* __restrict__ L, double* __restrict__ Xi, int K,
-                                                         int b) {
+// Xi = L^-1 (L lower, the factored Hr), right-looking over block rows; Xi starts at zero and its rows below the
+// current one accumulate T[i][c] = sum_{k < i} L[i][k] Xi[k][c].
+// Row k: CTA c (0 .. k) solves L[k][k] Xi[k][c] = (c == k ? I : -T[k][c]) by forward substitution.
+__global__ void __launch_bounds__(256) trtri_solve_kernel(const double* __restrict__ L, double* __restrict__ Xi, int K,
+                                                           int k) {
   extern __shared__ double tsm[];
-  double* La = tsm;                   // [64][65]
-  double* Xb = La + kT * (kT + 1);    // [64][65]
-  double* T = Xb + kT * (kT + 1);     // [64][65]
+  double* La = tsm;                 // [64][65] the diagonal tile L[k][k]
+  double* T = La + kT * (kT + 1);   // [64][65] right-hand side, then the solution
   const int c = blockIdx.x, tid = threadIdx.x;
-  const int ty = tid / 16, tx = tid % 16;
-  double acc[4][4] = {};
-  for (int k = c; k < b; ++k) {
-    for (int e = tid; e < kT * kT; e += 256) {
-      const int r = e / kT, q = e % kT;
-      La[r * (kT + 1) + q] = L[(size_t)(b * kT + r) * K + k * kT + q];
-      Xb[r * (kT + 1) + q] = Xi[(size_t)(k * kT + r) * K + c * kT + q];
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int q = 0; q < kT; ++q)
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          acc[u][v] = fma(La[(ty + 16 * u) * (kT + 1) + q], Xb[q * (kT + 1) + tx + 16 * v], acc[u][v]);
-    __syncthreads();
+  for (int e = tid; e < kT * kT; e += 256) {
+    const int r = e / kT, q = e % kT;
+    La[r * (kT + 1) + q] = L[(size_t)(k * kT + r) * K + k * kT + q];
+    T[r * (kT + 1) + q] = (c == k) ? (r == q ? 1.0 : 0.0) : -Xi[(size_t)(k * kT + r) * K + c * kT + q];
   }
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int r = ty + 16 * u, s = tx + 16 * v;
-      T[r * (kT + 1) + s] = (c == b) ? (r == s ? 1.0 : 0.0) : -acc[u][v];
-    }
-  for (int e = tid; e < kT * kT; e += 256)  // the diagonal tile L[b][b]
-    La[(e / kT) * (kT + 1) + e % kT] = L[(size_t)(b * kT + e / kT) * K + b * kT + e % kT];
   __syncthreads();
-  if (tid < kT) {  // column tid of the right-hand side, forward substitution down the rows
+  if (tid < kT) {  // column tid of the right-hand side, down the rows
     for (int r = 0; r < kT; ++r) {
       double v = T[r * (kT + 1) + tid];
       for (int q = 0; q < r; ++q) v -= La[r * (kT + 1) + q] * T[q * (kT + 1) + tid];
@@ -210,7 +189,41 @@ __global__ void __launch_bounds__(256) trtri_row_kernel(const double* __restrict
   }
   __syncthreads();
   for (int e = tid; e < kT * kT; e += 256)
-    Xi[(size_t)(b * kT + e / kT) * K + c * kT + e % kT] = T[(e / kT) * (kT + 1) + e % kT];
+    Xi[(size_t)(k * kT + e / kT) * K + c * kT + e % kT] = T[(e / kT) * (kT + 1) + e % kT];
+}
+
+// After row k: T[i][c] += L[i][k] Xi[k][c] for every later row block i > k and column block c <= k (one tile per
+// CTA; the later rows' accumulators live in Xi until their own solve).
+__global__ void __launch_bounds__(256) trtri_update_kernel(const double* __restrict__ L, double* __restrict__ Xi, int K,
+                                                            int k) {
+  __shared__ double La[kT][33];
+  __shared__ double Xb[32][kT + 1];
+  const int cols = k + 1;
+  const int i = k + 1 + blockIdx.x / cols, c = blockIdx.x % cols;
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[4][4] = {};
+  for (int q0 = 0; q0 < kT; q0 += 32) {
+    for (int e = threadIdx.x; e < kT * 32; e += 256) {
+      const int r = e / 32, q = e % 32;
+      La[r][q] = L[(size_t)(i * kT + r) * K + k * kT + q0 + q];
+    }
+    for (int e = threadIdx.x; e < 32 * kT; e += 256) {
+      const int q = e / kT, col = e % kT;
+      Xb[q][col] = Xi[(size_t)(k * kT + q0 + q) * K + c * kT + col];
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int q = 0; q < 32; ++q)
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fma(La[ty + 16 * u][q], Xb[q][tx + 16 * v], acc[u][v]);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) Xi[(size_t)(i * kT + ty + 16 * u) * K + c * kT + tx + 16 * v] += acc[u][v];
 }
 
 struct GptqParams {
@@ -381,8 +394,8 @@ bool attrs_set() {
     if (cudaFuncSetAttribute(gptq_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)gptq_block_smem()) != cudaSuccess)
       return false;
-    if (cudaFuncSetAttribute(trtri_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(3 * kT * (kT + 1) * sizeof(double))) != cudaSuccess)
+    if (cudaFuncSetAttribute(trtri_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(2 * kT * (kT + 1) * sizeof(double))) != cudaSuccess)
       return false;
     if (cudaFuncSetAttribute(chol_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(2 * kT * (kT + 1) * sizeof(double))) != cudaSuccess)
@@ -430,9 +443,11 @@ awq_status gptq_launch(const uint16_t* W, const uint16_t* xcal, int N, int K, in
     chol_update_kernel<<<m * (m + 1) / 2 + 1, 256, 0, st>>>(Hr, K, c, D);
     if (cudaGetLastError() != cudaSuccess) return AWQ_ERR_CUDA;
   }
-  const size_t tri_smem = 3 * kT * (kT + 1) * sizeof(double);
-  for (int b = 0; b < nb; ++b) {
-    trtri_row_kernel<<<b + 1, 256, tri_smem, st>>>(Hr, Xi, K, b);
+  const size_t tri_smem = 2 * kT * (kT + 1) * sizeof(double);
+  if (cudaMemsetAsync(Xi, 0, (size_t)K * K * sizeof(double), st) != cudaSuccess) return AWQ_ERR_CUDA;
+  for (int k = 0; k < nb; ++k) {
+    trtri_solve_kernel<<<k + 1, 256, tri_smem, st>>>(Hr, Xi, K, k);
+    if (k + 1 < nb) trtri_update_kernel<<<(nb - k - 1) * (k + 1), 256, 0, st>>>(Hr, Xi, K, k);
     if (cudaGetLastError() != cudaSuccess) return AWQ_ERR_CUDA;
   }
   for (int b0 = 0; b0 < K; b0 += kGB) {

@@ -46,7 +46,7 @@ awq_status prep_inv_scale_launch(const uint16_t* x, const uint16_t* s, int M, in
 // (gate|up, N = 2 * NI, NI % 16 == 0): row 32j + i of the packed weight is W[16j + i] for i < 16 and
 // W2[16j + i - 16] for i >= 16.
 awq_status pack_launch(const uint16_t* W, const uint16_t* W2, const uint16_t* s, int N, int K, int g, uint32_t* qw,
-                       uint16_t* scales, uint32_t* qz, cudaStream_t st);
+                       uint16_t* scales, uint32_t* qz, cudaStream_t st, int w_bit = 4);
 
 // One linear-layer call as the kernels see it.
 struct LinearArgs {

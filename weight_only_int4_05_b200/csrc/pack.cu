@@ -4,9 +4,10 @@
 // Sources: "AWQ and GPTQ algorithms" (jsqmd.com), section 2.1 (3) (multiply the weight channels by s);
 // "LLM-AWQ academic impact" (CSDN mirror), "quantization flow" (w_bit 4, q_group_size 128, the real
 // quantization stage); "LLM quantization speed-up" (bjdmk.com.cn), "quantization parameters" (zero point).
-// Grid, in IEEE fp32 with correctly rounded operations and no contraction:
-//   w' = W*s; sc32 = max((max-min)/15, 1e-5); S = float(fp16(sc32)); z = clamp(rint(-min/S), 0, 15);
-//   q = clamp(rint(w'/S) + z, 0, 15).
+// Grid, in IEEE fp32 with correctly rounded operations and no contraction (qmax = 2^w_bit - 1: 15 for the
+// pages' 4 bits, 7 for the 3-bit grid, whose codes are stored in the same 4-bit layout):
+//   w' = W*s; sc32 = max((max-min)/qmax, 1e-5); S = float(fp16(sc32)); z = clamp(rint(-min/S), 0, qmax);
+//   q = clamp(rint(w'/S) + z, 0, qmax).
 //
 // One CTA per run of kPackGroups units of one row block (the units (rb, g0 .. g0+3) are consecutive in all
 // three packed arrays).  LPG = GS / 8 lanes take one (row, group): lane h of them holds channels 8h..8h+7
@@ -25,12 +26,12 @@ namespace awq {
 
 constexpr int kPackGroups = 4;  // units per CTA
 
-__device__ __forceinline__ float clamp015(float v) { return fminf(fmaxf(v, 0.0f), 15.0f); }
+__device__ __forceinline__ float clamp0q(float v, float qmax) { return fminf(fmaxf(v, 0.0f), qmax); }
 __device__ __forceinline__ float h2f_bits(uint32_t bits) { return __half2float(__ushort_as_half((unsigned short)bits)); }
 
 template <int GS>
 __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W, const __half* __restrict__ W2,
-                                                    const __half* __restrict__ s, int N, int K, int G,
+                                                    const __half* __restrict__ s, int N, int K, int G, float qmax,
                                                     uint8_t* __restrict__ qw, uint16_t* __restrict__ scales,
                                                     uint32_t* __restrict__ qz) {
   // No griddepcontrol.launch_dependents here: the linear kernels read packed weights before their own
@@ -91,14 +92,14 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
         mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
         mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
       }
-      const float sc32 = fmaxf(__fdiv_rn(__fsub_rn(mx, mn), 15.0f), 1e-5f);
+      const float sc32 = fmaxf(__fdiv_rn(__fsub_rn(mx, mn), qmax), 1e-5f);
       const __half sch = __float2half_rn(sc32);
       const float S = __half2float(sch);
-      const float zf = clamp015(rintf(__fdiv_rn(-mn, S)));
+      const float zf = clamp0q(rintf(__fdiv_rn(-mn, S)), qmax);
       uint32_t word = 0u;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const uint32_t code = (uint32_t)(int)clamp015(__fadd_rn(rintf(__fdiv_rn(wp[e], S)), zf));
+        const uint32_t code = (uint32_t)(int)clamp0q(__fadd_rn(rintf(__fdiv_rn(wp[e], S)), zf), qmax);
         word |= code << (4 * ((e & 1) ? 4 + (e >> 1) : (e >> 1)));
       }
       // word hl & 3 of row r in the unit's chunk hl >> 2 (chunk = 512 B = 128 words, row = 4 words)
@@ -124,7 +125,8 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half* __restrict__ W,
 }
 
 awq_status pack_launch(const uint16_t* W, const uint16_t* W2, const uint16_t* s, int N, int K, int g, uint32_t* qw,
-                       uint16_t* scales, uint32_t* qz, cudaStream_t st) {
+                       uint16_t* scales, uint32_t* qz, cudaStream_t st, int w_bit) {
+  const float qmax = (float)((1 << w_bit) - 1);
   const int RB = (N + 31) / 32;
   const int G = K / g;
   const dim3 grid((unsigned)RB, (unsigned)((G + kPackGroups - 1) / kPackGroups));  // x: row blocks (no 65535 cap)
@@ -134,9 +136,9 @@ awq_status pack_launch(const uint16_t* W, const uint16_t* W2, const uint16_t* s,
   uint8_t* q = reinterpret_cast<uint8_t*>(qw);
   cudaError_t e;
   switch (g) {
-    case 64: e = launch_pdl(pack_kernel<64>, grid, dim3(256), 0, st, w, w2, sh, N, K, G, q, scales, qz); break;
-    case 256: e = launch_pdl(pack_kernel<256>, grid, dim3(256), 0, st, w, w2, sh, N, K, G, q, scales, qz); break;
-    default: e = launch_pdl(pack_kernel<128>, grid, dim3(256), 0, st, w, w2, sh, N, K, G, q, scales, qz); break;
+    case 64: e = launch_pdl(pack_kernel<64>, grid, dim3(256), 0, st, w, w2, sh, N, K, G, qmax, q, scales, qz); break;
+    case 256: e = launch_pdl(pack_kernel<256>, grid, dim3(256), 0, st, w, w2, sh, N, K, G, qmax, q, scales, qz); break;
+    default: e = launch_pdl(pack_kernel<128>, grid, dim3(256), 0, st, w, w2, sh, N, K, G, qmax, q, scales, qz); break;
   }
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
