@@ -424,3 +424,66 @@ out:
   free(H); free(U); free(Wc); free(E); free(gv); free(S); free(zz); free(gx);
   return rc;
 }
+
+/* ------------------------------------------------------------------------------------------------ */
+/* The packed 3-bit layout (the public header's prose, "3-BIT LAYOUT"): per 32-row block rb, 32-channel
+ * chunk kc and row r, three 32-bit words at word (rb * (K/32) + kc) * 96 + 3 r:
+ *   word 0: the low 2 bits of channels 0..15 of the chunk, word 1: of channels 16..31.  Channel 8j + 2p + h
+ *           (j = 0..3 the 8-channel group, p = 0..3 the pair, h = 0..1) sits at bit 8 (j % 2) + 2p + 16h of
+ *           word j / 2;
+ *   word 2: the high bit of channel 8j + 2p + h at bit 4j + p + 16h.
+ * Scales and zeros: exactly as the 4-bit layout (unit major, 64 B and 16 B per unit).                   */
+void oracle_pack3(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int N, int K, int g,
+                  uint32_t* qweight, uint16_t* scales, uint32_t* qzeros) {
+  int G = K / g;
+  int Np = round_up32(N);
+  int KC = K / 32;
+  memset(qweight, 0, sizeof(uint32_t) * (size_t)Np * KC * 3);
+  memset(scales, 0, sizeof(uint16_t) * (size_t)G * Np);
+  memset(qzeros, 0, sizeof(uint32_t) * (size_t)G * Np / 8);
+  for (int n = 0; n < N; ++n) {
+    int rb = n / 32, r = n % 32;
+    for (int k = 0; k < K; ++k) {
+      int kc = k / 32, c = k % 32, j = c / 8, p = (c % 8) / 2, h = c % 2;
+      uint32_t code = q[(size_t)n * K + k] & 7u;
+      size_t base = ((size_t)rb * KC + kc) * 96 + (size_t)r * 3;
+      qweight[base + (size_t)(j / 2)] |= (code & 3u) << (8 * (j % 2) + 2 * p + 16 * h);
+      qweight[base + 2] |= (code >> 2) << (4 * j + p + 16 * h);
+    }
+    for (int gi = 0; gi < G; ++gi) {
+      size_t unit = (size_t)rb * G + gi;
+      scales[unit * 32 + r] = sc[(size_t)n * G + gi];
+      qzeros[unit * 4 + r / 8] |= (uint32_t)(z[(size_t)n * G + gi] & 0xF) << (4 * (r % 8));
+    }
+  }
+}
+
+/* Independent decoder of the 3-bit layout: walks every stored word and asks which (row, channel) each of
+ * its bits belongs to. */
+void oracle_unpack3(const uint32_t* qweight, int N, int K, uint8_t* q) {
+  int Np = round_up32(N);
+  int KC = K / 32;
+  size_t nwords = (size_t)Np * KC * 3;
+  memset(q, 0, (size_t)N * K);
+  for (size_t w = 0; w < nwords; ++w) {
+    size_t tile = w / 96;
+    int within = (int)(w % 96), r = within / 3, kind = within % 3;
+    int rb = (int)(tile / (size_t)KC), kc = (int)(tile % (size_t)KC);
+    int n = rb * 32 + r;
+    if (n >= N) continue;
+    for (int bit = 0; bit < 32; ++bit) {
+      uint32_t v = (qweight[w] >> bit) & 1u;
+      int h = bit / 16, b = bit % 16, c, shift;
+      if (kind < 2) { /* low bits: b = 8 (j % 2) + 2p + t, t the bit of the 2-bit field */
+        int jj = b / 8, p = (b % 8) / 2, t = b % 2;
+        c = 8 * (2 * kind + jj) + 2 * p + h;
+        shift = t;
+      } else { /* high bit: b = 4j + p */
+        int j = b / 4, p = b % 4;
+        c = 8 * j + 2 * p + h;
+        shift = 2;
+      }
+      q[(size_t)n * K + kc * 32 + c] |= (uint8_t)(v << shift);
+    }
+  }
+}

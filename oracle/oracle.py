@@ -63,6 +63,8 @@ def _load():
             lib.oracle_inv_scale.argtypes = [P, P, I, I, P]
             lib.oracle_quantize.argtypes = [P, P, I, I, I, P, P, P]
             lib.oracle_quantize_bits.argtypes = [P, P, I, I, I, I, P, P, P]
+            lib.oracle_pack3.argtypes = [P, P, P, I, I, I, P, P, P]
+            lib.oracle_unpack3.argtypes = [P, I, I, P]
             lib.oracle_pack.argtypes = [P, P, P, I, I, I, P, P, P]
             lib.oracle_unpack.argtypes = [P, P, P, I, I, I, P, P, P]
             lib.oracle_dequant.argtypes = [P, P, P, I, I, I, P]
@@ -70,7 +72,8 @@ def _load():
             lib.oracle_linear_pairs_f64.argtypes = [P, P, P, P, I, I, I, I, P, P, I, P]
             for name in ("oracle_act_scale", "oracle_inv_scale", "oracle_quantize", "oracle_pack",
                          "oracle_unpack", "oracle_dequant", "oracle_linear_f64", "oracle_linear_pairs_f64",
-                         "oracle_act_pow", "oracle_f64_to_f16_array", "oracle_quantize_bits"):
+                         "oracle_act_pow", "oracle_f64_to_f16_array", "oracle_quantize_bits", "oracle_pack3",
+                         "oracle_unpack3"):
                 getattr(lib, name).restype = None
             _lib = lib
     return _lib
@@ -332,3 +335,35 @@ def gptq_quantize(W, xcal, g: int = GROUP, damp: float = GPTQ_DAMP):
     if _load().oracle_gptq(_p(W), _p(xcal), N, K, R, g, ctypes.c_double(damp), _p(q), _p(sc), _p(z)) != 0:
         raise ValueError("the Hessian is not positive definite")
     return q, sc, z
+
+
+
+# ---- the packed 3-bit layout -----------------------------------------------------------------------
+def packed3_sizes(N: int, K: int, g: int = GROUP):
+    """Bytes of (qweight, scales, qzeros) in the 3-bit layout: 12 bytes per row per 32 channels."""
+    Np = (N + 31) // 32 * 32
+    G = K // g
+    return Np * K // 32 * 12, G * Np * 2, G * Np // 2
+
+
+def pack3(q, sc, z, g: int = GROUP):
+    N, K = q.shape
+    Np = (N + 31) // 32 * 32
+    G = K // g
+    qw = np.empty(Np * K // 32 * 3, np.uint32)
+    scales = np.empty(G * Np, np.uint16)
+    qz = np.empty(G * Np // 8, np.uint32)
+    _load().oracle_pack3(_p(np.ascontiguousarray(q)), _p(np.ascontiguousarray(sc)), _p(np.ascontiguousarray(z)),
+                         N, K, g, _p(qw), _p(scales), _p(qz))
+    return qw, scales, qz
+
+
+def unpack3(qw, N: int, K: int) -> np.ndarray:
+    q = np.empty((N, K), np.uint8)
+    _load().oracle_unpack3(_p(np.ascontiguousarray(qw)), N, K, _p(q))
+    return q
+
+
+def awq_pack3(W, s=None, g: int = GROUP):
+    """Quantize on the 3-bit grid and pack into the 3-bit layout: (qweight, scales, qzeros)."""
+    return pack3(*quantize(W, s, g, 3), g)

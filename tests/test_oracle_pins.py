@@ -797,3 +797,58 @@ def test_quantize_3bit_clamps_and_bound():
     assert np.mean((deq3 - wp) ** 2) > 3.0 * np.mean((deq4 - wp) ** 2)
     for a, b in zip(O.quantize(W, s, 128, 4), O.quantize(W, s)):
         assert np.array_equal(a, b)  # w_bit = 4 is the default grid
+
+
+# ---------------------------------------------------------------- packed 3-bit layout --------------
+def _expected3(n, k, K):
+    """(word index, bit) of the low 2 bits and of the high bit of (n, k), read off the header's prose."""
+    rb, r, kc, c = n // 32, n % 32, k // 32, k % 32
+    j, p, h = c // 8, (c % 8) // 2, c % 2
+    base = (rb * (K // 32) + kc) * 96 + 3 * r
+    return (base + j // 2, 8 * (j % 2) + 2 * p + 16 * h), (base + 2, 4 * j + p + 16 * h)
+
+
+def test_pack3_single_code_placement():
+    """A single nonzero 3-bit code lands at the two words and bits the header describes."""
+    N, K = 40, 256
+    rng = np.random.default_rng(83)
+    for _ in range(80):
+        n, k, c = int(rng.integers(N)), int(rng.integers(K)), int(rng.integers(1, 8))
+        q = np.zeros((N, K), np.uint8)
+        q[n, k] = c
+        qw, _, _ = O.pack3(q, np.zeros((N, 2), np.uint16), np.zeros((N, 2), np.uint8))
+        (wl, bl), (wh, bh) = _expected3(n, k, K)
+        exp = np.zeros_like(qw)
+        exp[wl] |= (c & 3) << bl
+        exp[wh] |= (c >> 2) << bh
+        assert np.array_equal(qw, exp)
+
+
+def test_pack3_sizes_roundtrip_and_extraction():
+    """3 words per row per 32 channels (0.375 B per weight of codes); the independent decoder inverts the
+    packer; and the extraction the header promises: for lane group j and pair p, the low bits of channels
+    (8j + 2p, 8j + 2p + 1) are (word_{j/2} >> (8 (j%2) + 2p)) & 0x00030003, their high bits
+    (word_2 >> (4j + p)) & 0x00010001."""
+    rng = np.random.default_rng(89)
+    N, K = 72, 384
+    q = rng.integers(0, 8, (N, K)).astype(np.uint8)
+    sc = rng.integers(1, 0x7BFF, (N, 3)).astype(np.uint16)
+    z = rng.integers(0, 8, (N, 3)).astype(np.uint8)
+    qw, scales, qz = O.pack3(q, sc, z)
+    assert (qw.nbytes, scales.nbytes, qz.nbytes) == O.packed3_sizes(N, K)
+    assert qw.nbytes == 96 * (K // 32) * 12  # N_pad = 96 rows x 12 B per 32 channels
+    assert np.array_equal(O.unpack3(qw, N, K), q)
+    qw4, scales4, qz4 = O.pack(q, sc, z)
+    assert np.array_equal(scales, scales4) and np.array_equal(qz, qz4)  # scales and zeros as the 4-bit layout
+    for n in range(0, N, 7):
+        rb, r = n // 32, n % 32
+        for kc in range(K // 32):
+            base = (rb * (K // 32) + kc) * 96 + 3 * r
+            w = [int(qw[base + i]) for i in range(3)]
+            for j in range(4):
+                for p in range(4):
+                    lo = (w[j // 2] >> (8 * (j % 2) + 2 * p)) & 0x00030003
+                    hi = (w[2] >> (4 * j + p)) & 0x00010001
+                    c0, c1 = q[n, kc * 32 + 8 * j + 2 * p], q[n, kc * 32 + 8 * j + 2 * p + 1]
+                    assert (lo & 0xFFFF) | ((hi & 0xFFFF) << 2) == c0
+                    assert (lo >> 16) | ((hi >> 16) << 2) == c1
