@@ -627,6 +627,35 @@ def measure_groups(device, peaks, reps):
     return out
 
 
+def measure_int3(device, peaks, reps):
+    """The packed 3-bit layout: the M=1 decode shapes through w3a16_gemv (calls over weight copies larger than
+    L2, one graph); bytes counted at 0.375 + 2.5/128 per weight."""
+    import torch
+    import synth
+    import weight_only_int4_05_b200 as W4
+
+    out = []
+    for i, (name, K, N) in enumerate([("q/o", 4096, 4096), ("k/v", 4096, 1024), ("gate/up", 4096, 14336),
+                                      ("down", 14336, 4096)]):
+        Wt, xcal, x = synth.device_linear_inputs(0, synth.tensor_id(1, 0, i, 0), 1, N, K, device)
+        s = W4.awq_act_scale(xcal)
+        xp = W4.awq_apply_inv_scale(x, s)
+        per = N * K * (0.375 + 2.5 / 128)
+        pws = [W4.awq_pack3(Wt, s) for _ in range(max(2, int(-(-(512 * 2**20) // per))))]
+        del Wt, xcal, x
+        y = torch.empty((1, N), dtype=torch.float16, device=device)
+        ws = W4.reserve_workspace(max(256, W4.w4a16_workspace_bytes(W4.MODE_GEMV, 1, N, K)), device)
+        calls = [(lambda p=pw: W4.w3a16_gemv(xp, p, out=y, workspace=ws)) for pw in pws]
+        sec = time_graph_calls(calls, reps, 3, device)
+        b = per + 2 * K + 2 * N
+        out.append({"shape": name, "K": K, "N": N, "M": 1, "us": round(sec * 1e6, 3),
+                    "GB/s": round(b / sec / 1e9, 1), "frac": round(b / sec / 1e9 / peaks["hbm_gbs"], 4),
+                    "weights_per_s_G": round(N * K / sec / 1e9, 1)})
+        del pws
+        torch.cuda.empty_cache()
+    return out
+
+
 def measure_search(device, reps=3):
     """awq_search_scale on the 4096 -> 4096 projection with 512 calibration rows and 21 grid points, device
     time per search through the C entry point (preallocated buffers; no host synchronisation inside)."""
@@ -850,6 +879,7 @@ def run_gpu(args):
     pack = measure_pack(device, peaks, reps)
     crossover = None if args.no_crossover else measure_crossover(device, max(3, reps // 4))
     groups = measure_groups(device, peaks, reps)
+    int3 = measure_int3(device, peaks, reps)
     search = measure_search(device)
     gptq = measure_gptq(device)
 
@@ -868,7 +898,8 @@ def run_gpu(args):
                     "steps": e2e_steps},
             "gemm": gemm, "decode_sweep": sweep, "tiny": tiny, "pack": pack, "crossover": crossover,
             "decode_prefetch_hint": decode_pf, "decode_fused": decode_fused, "decode_inv_s_fused": decode_inv_s,
-            "decode_fused_silu": decode_fused_silu, "group_sizes": groups, "awq_search": search, "gptq": gptq}
+            "decode_fused_silu": decode_fused_silu, "group_sizes": groups, "int3_layout": int3, "awq_search": search,
+            "gptq": gptq}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     elif rank == 0:

@@ -65,6 +65,18 @@
  *   Padding rows n = N .. N_pad-1 hold code 0, scale 0 and zero 0 in every array.
  *   Bytes per weight (N a multiple of 32): 0.5 + 2.5/g = 0.51953 at g = 128 (0.53906 at 64, 0.50977 at 256).
  *
+ * 3-BIT LAYOUT (awq_pack3; read by w3a16_gemv): the same row blocks, 32-channel chunks, units, scales and
+ * zeros as above, with 12 bytes per row per chunk instead of 16:
+ *   qweight  uint32_t[N_pad * K / 32 * 3].  Tile (rb, kc) is 384 contiguous bytes, 32 rows x 3 words, row r's
+ *            words at word offset (rb * (K/32) + kc) * 96 + 3 r.  For channel c = 8j + 2p + h of the chunk
+ *            (j = 0..3 the 8-channel group, p = 0..3 the pair, h = 0..1 the half) with 3-bit code q:
+ *              word j / 2 holds q & 3 at bits 8 (j % 2) + 2p + 16h .. +1   (the low 2-bit plane),
+ *              word 2 holds q >> 2 at bit 4j + p + 16h                     (the high-bit plane).
+ *            So for group j and pair p, ((word_{j/2} >> (8 (j%2) + 2p)) & 0x00030003) | ((word_2 >> (4j + p))
+ *            & 0x00010001) << 2 puts the codes of channels 8j + 2p and 8j + 2p + 1 in the two 16-bit halves.
+ *            A unit (32 rows x g channels) is 12 g contiguous bytes.  Bytes per weight: 0.375 + 2.5/g
+ *            (0.39453 at g = 128, 24 % less than the 4-bit layout).
+ *
  * QUANTIZATION GRID (what awq_pack computes; plain reading of [AutoAWQ] zero point + [LLM-AWQ] w_bit 4,
  * q_group_size g as asymmetric min/max round-to-nearest), per row n and group gi, all in IEEE fp32
  * with correctly rounded operations and no fused multiply-add:
@@ -161,6 +173,27 @@ awq_status awq_pack(const uint16_t* d_W, const uint16_t* d_s, int N, int K, int 
  */
 awq_status awq_pack_bits(const uint16_t* d_W, const uint16_t* d_s, int N, int K, int g, int w_bit, uint32_t* d_qweight,
                          uint16_t* d_scales, uint32_t* d_qzeros, awq_stream_t stream);
+
+/* awq_packed3_sizes -- byte sizes of the three arrays of the 3-bit layout (above) for an N x K weight at g. */
+awq_status awq_packed3_sizes(int N, int K, int g, size_t* qweight_bytes, size_t* scales_bytes, size_t* qzeros_bytes);
+
+/*
+ * awq_pack3 -- awq_pack on the 3-bit grid (qmax = 7; awq_pack_bits with w_bit = 3) written in the packed 3-bit
+ * layout ([LLM-AWQ] "choose 4-bit or 3-bit quantization by hardware resources"; [INT4-VLM] introduction, AWQ at
+ * INT3): 0.39 bytes per weight.  Arguments and errors as awq_pack; outputs sized by awq_packed3_sizes.
+ */
+awq_status awq_pack3(const uint16_t* d_W, const uint16_t* d_s, int N, int K, int g, uint32_t* d_qweight,
+                     uint16_t* d_scales, uint32_t* d_qzeros, awq_stream_t stream);
+
+/*
+ * w3a16_gemv -- the decode kernel of w4a16_gemv on a weight from awq_pack3: the same plans, warp roles, tensor-core
+ * contraction (exact q - z products, fp32 sums) and epilogue, with each unit's codes read from the 3-bit layout.
+ * Any M (passes of up to 16 rows).  Arguments, workspace (w4a16_workspace_bytes(AWQ_MODE_GEMV, ...)) and errors
+ * as w4a16_gemv.  There is no 3-bit GEMM: prefill-sized M runs here, in passes.
+ */
+awq_status w3a16_gemv(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                      const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g, void* d_workspace,
+                      size_t workspace_bytes, awq_stream_t stream);
 
 /*
  * awq_pack_gate_up -- packs the gate and up projections of a gated MLP (both [NI][K], the same input x)

@@ -173,3 +173,15 @@ def test_pack_bits_argument_checks(L):
     assert L.awq_pack_bits(F, None, 256, 512, 128, 2, F, F, F, None) == 2
     assert L.awq_pack_bits(F, None, 256, 500, 128, 3, F, F, F, None) == 1   # K % g != 0
     assert L.awq_pack_bits(P(FAKE + 8), None, 256, 512, 128, 3, F, F, F, None) == 3
+
+
+def test_three_bit_layout_sizes_and_checks(L):
+    P, F = ctypes.c_void_p, ctypes.c_void_p(FAKE)
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.awq_packed3_sizes(40, 512, 128, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)) == 0
+    assert a.value == 64 * 512 // 32 * 12 and b.value == 4 * 64 * 2 and c.value == 4 * 64 // 2
+    assert L.awq_pack3(F, None, 256, 512, 32, F, F, F, None) == 2
+    assert L.awq_pack3(F, None, 256, 500, 128, F, F, F, None) == 1
+    assert L.awq_pack3(P(FAKE + 8), None, 256, 512, 128, F, F, F, None) == 3
+    assert L.w3a16_gemv(F, F, F, F, F, 0, 256, 512, 128, None, 0, None) == 1
+    assert L.w3a16_gemv(F, F, F, F, F, 1, 256, 512, 32, None, 0, None) == 2

@@ -38,6 +38,7 @@ class PackedWeight(NamedTuple):
     N: int
     K: int
     g: int = GROUP          # group size the weight was packed with
+    bits: int = 4           # code layout: 4 (w4a16_* calls) or 3 (awq_pack3 / w3a16_gemv)
 
 
 class SearchResult(NamedTuple):
@@ -177,7 +178,9 @@ def reserve_workspace(nbytes: int, device=None) -> torch.Tensor:
     return ws
 
 
-def _group(pw: PackedWeight, g: Optional[int]) -> int:
+def _group(pw: PackedWeight, g: Optional[int], bits: int = 4) -> int:
+    if pw.bits != bits:
+        raise ValueError(f"the weight has the {pw.bits}-bit layout; this call reads the {bits}-bit layout")
     if g is not None and g != pw.g:
         raise ValueError(f"g={g} but the weight was packed with g={pw.g}")
     return pw.g
@@ -343,3 +346,42 @@ def gptq_quantize(W: torch.Tensor, xcal: torch.Tensor, g: int = GROUP, damp: flo
                          ws.numel() * ws.element_size(), _stream(dev))
     _lib.check(st, "gptq_quantize")
     return PackedWeight(qw, sc, qz, N, K, g)
+
+
+def awq_pack3(W: torch.Tensor, s: Optional[torch.Tensor] = None, g: int = GROUP) -> PackedWeight:
+    """Quantizes W (s folded in) on the 3-bit grid into the packed 3-bit layout (0.39 B per weight), for
+    w3a16_gemv."""
+    _need_cuda_fp16(W, "W")
+    N, K = W.shape
+    if s is not None:
+        _need_cuda_fp16(s, "s")
+        if s.shape != (K,):
+            raise ValueError(f"s has shape {tuple(s.shape)}, expected ({K},)")
+    L = _lib.load()
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _lib.check(L.awq_packed3_sizes(N, K, g, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)), "awq_packed3_sizes")
+    dev = W.device
+    qw = torch.empty(a.value // 4, dtype=torch.int32, device=dev)
+    sc = torch.empty(b.value // 2, dtype=torch.float16, device=dev)
+    qz = torch.empty(c.value // 4, dtype=torch.int32, device=dev)
+    _lib.check(L.awq_pack3(_p(W), _p(s), N, K, g, _p(qw), _p(sc), _p(qz), _stream(dev)), "awq_pack3")
+    return PackedWeight(qw, sc, qz, N, K, g, 3)
+
+
+def w3a16_gemv(x, pw: PackedWeight, out=None, workspace=None) -> torch.Tensor:
+    """The decode GEMV on a weight from awq_pack3 (any M, in passes of up to 16 rows)."""
+    _need_cuda_fp16(x, "x")
+    g = _group(pw, None, 3)
+    M, K = x.shape
+    if K != pw.K:
+        raise ValueError(f"x has K={K}, weight has K={pw.K}")
+    N = pw.N
+    if out is not None:
+        _check_out(out, (M, N), x.device)
+    y = torch.empty((M, N), dtype=torch.float16, device=x.device) if out is None else out
+    need = w4a16_workspace_bytes(MODE_GEMV, M, N, K, g)
+    ws = workspace if workspace is not None else (reserve_workspace(need, x.device) if need > 0 else None)
+    st = _lib.load().w3a16_gemv(_p(x), _p(pw.qweight), _p(pw.scales), _p(pw.qzeros), _p(y), M, N, K, g, _p(ws),
+                                0 if ws is None else ws.numel() * ws.element_size(), _stream(x.device))
+    _lib.check(st, "w3a16_gemv")
+    return y

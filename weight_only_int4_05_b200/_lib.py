@@ -15,7 +15,8 @@ EXPORTS = (
     "awq_pack", "w4a16_gemv", "w4a16_gemm", "w4a16_linear", "w4a16_gemv_max_m", "w4a16_workspace_bytes",
     "awq_last_device_status", "w4a16_gemv_noalloc", "awq_selftest_wait_timeout",
     "w4a16_linear_pf", "w4a16_gemv_s", "awq_pack_gate_up", "w4a16_gate_up_silu", "awq_search_scale",
-    "awq_search_workspace_bytes", "gptq_quantize", "gptq_workspace_bytes", "awq_pack_bits",
+    "awq_search_workspace_bytes", "gptq_quantize", "gptq_workspace_bytes", "awq_pack_bits", "awq_packed3_sizes",
+    "awq_pack3", "w3a16_gemv",
 )
 
 STATUS_NAMES = {0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_UNSUPPORTED", 3: "AWQ_ERR_MISALIGNED",
@@ -58,6 +59,12 @@ def load() -> ctypes.CDLL:
         lib.awq_apply_inv_scale.argtypes = [P, P, I, I, P, P]
         lib.awq_pack.restype = I
         lib.awq_pack.argtypes = [P, P, I, I, I, P, P, P, P]
+        lib.awq_packed3_sizes.restype = I
+        lib.awq_packed3_sizes.argtypes = [I, I, I, ctypes.POINTER(Z), ctypes.POINTER(Z), ctypes.POINTER(Z)]
+        lib.awq_pack3.restype = I
+        lib.awq_pack3.argtypes = [P, P, I, I, I, P, P, P, P]
+        lib.w3a16_gemv.restype = I
+        lib.w3a16_gemv.argtypes = [P, P, P, P, P, I, I, I, I, P, Z, P]
         lib.awq_pack_bits.restype = I
         lib.awq_pack_bits.argtypes = [P, P, I, I, I, I, P, P, P, P]
         lib.gptq_quantize.restype = I

@@ -125,6 +125,26 @@ awq_status awq_pack_bits(const uint16_t* d_W, const uint16_t* d_s, int N, int K,
                      w_bit);
 }
 
+awq_status awq_packed3_sizes(int N, int K, int g, size_t* qweight_bytes, size_t* scales_bytes, size_t* qzeros_bytes) {
+  awq_status st = awq_packed_sizes(N, K, g, qweight_bytes, scales_bytes, qzeros_bytes);
+  if (st != AWQ_OK) return st;
+  if (K % 32 != 0) return AWQ_ERR_INVALID_ARG;
+  *qweight_bytes = *qweight_bytes / 4 * 3;  // 12 bytes per row per 32 channels instead of 16
+  return AWQ_OK;
+}
+
+awq_status awq_pack3(const uint16_t* d_W, const uint16_t* d_s, int N, int K, int g, uint32_t* d_qweight,
+                     uint16_t* d_scales, uint32_t* d_qzeros, awq_stream_t stream) {
+  if (!group_supported(g)) return AWQ_ERR_UNSUPPORTED;
+  if (N < 1 || K < g || K % g != 0 || N > kMaxN || K > kMaxK) return AWQ_ERR_INVALID_ARG;
+  if (!d_W || !d_qweight || !d_scales || !d_qzeros) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(d_W) || (d_s && !aligned16(d_s)) || !aligned16(d_qweight) || !aligned16(d_scales) ||
+      !aligned16(d_qzeros))
+    return AWQ_ERR_MISALIGNED;
+  return pack_launch(d_W, nullptr, d_s, N, K, g, d_qweight, d_scales, d_qzeros, reinterpret_cast<cudaStream_t>(stream),
+                     3, 3);
+}
+
 awq_status awq_pack_gate_up(const uint16_t* d_Wgate, const uint16_t* d_Wup, const uint16_t* d_s, int NI, int K, int g,
                             uint32_t* d_qweight, uint16_t* d_scales, uint32_t* d_qzeros, awq_stream_t stream) {
   if (!group_supported(g)) return AWQ_ERR_UNSUPPORTED;
@@ -262,6 +282,20 @@ awq_status w4a16_gate_up_silu(const uint16_t* d_x, const uint32_t* d_qweight, co
   if (M <= w4a16_gemv_max_m(N, K)) return gemv_launch(a);
   if (workspace_bytes < gemm_workspace_bytes(M, N, K, g)) return AWQ_ERR_WORKSPACE;
   return gemm_launch(a);
+}
+
+awq_status w3a16_gemv(const uint16_t* d_x, const uint32_t* d_qweight, const uint16_t* d_scales,
+                      const uint32_t* d_qzeros, uint16_t* d_y, int M, int N, int K, int g, void* d_workspace,
+                      size_t workspace_bytes, awq_stream_t stream) {
+  awq_status st = check_linear(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g);
+  if (st != AWQ_OK) return st;
+  if (d_workspace && !aligned16(d_workspace)) return AWQ_ERR_MISALIGNED;
+  unsigned* status = device_status_ptr();
+  if (status == nullptr) return AWQ_ERR_CUDA;
+  LinearArgs a = linear_args(d_x, d_qweight, d_scales, d_qzeros, d_y, M, N, K, g, d_workspace, workspace_bytes,
+                             status, stream);
+  a.bits = 3;
+  return gemv_launch(a);
 }
 
 static bool gptq_args_ok(int N, int K, int R, int g, double damp) {

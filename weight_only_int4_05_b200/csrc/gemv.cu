@@ -30,6 +30,9 @@
 // (even and odd chunks).  After the steps of a group the fp32 sum of each row is multiplied by the row's
 // scale and added to the row's fp32 output accumulator.  Nothing is summed in fp16.
 //
+// 3-bit codes (BITS = 3, the packed 3-bit layout): the same kernel with 384-B tiles and unit_mma3 building the
+// fp16 pairs from a 2-bit plane and a 1-bit plane.
+//
 // Epilogue.  Plain: y = fp16(sum).  Gate|up (epi = 1, the weight packed by awq_pack_gate_up, rows 0..15 of
 // row block j the gate rows 16j..16j+15 and rows 16..31 the up rows 16j..16j+15): the output has N / 2
 // columns, h[m][16j + i] = fp16(silu(sum of row i) * sum of row 16 + i), silu(a) = a / (1 + e^-a), in fp32
@@ -74,17 +77,22 @@ static_assert((kNW & (kNW - 1)) == 0 && kNW >= 2 && kNW <= 16, "consumer warps p
 constexpr int kSlots = kNW * kRing;
 constexpr int kThreads = (kNW + 1) * 32;
 
-// Geometry of a unit and a slot for group size GS.
-template <int GS>
+// Geometry of a unit and a slot for group size GS and code width BITS (4: the 4-bit layout, 512-B tiles of 32 rows
+// x 32 channels; 3: the packed 3-bit layout, 384-B tiles).  A slot holds 8 KB (6 KB at 3 bits) of codes: the
+// same number of units either way.
+template <int GS, int BITS = 4>
 struct Geo {
   static_assert(GS == 64 || GS == 128 || GS == 256, "group size 64, 128 or 256");
-  static constexpr int CH = GS / 32;                   // 32-channel chunks (512-B tiles) per unit
-  static constexpr int UB = 16 * GS;                   // code bytes per unit
-  static constexpr int SU = kSlotCodeBytes / UB;       // units per slot: 8, 4, 2
-  static constexpr int SCO = kSlotCodeBytes;           // scales offset in a slot
-  static constexpr int ZO = SCO + SU * 64;             // zeros offset in a slot
+  static_assert(BITS == 3 || BITS == 4, "3- or 4-bit codes");
+  static constexpr int CH = GS / 32;                    // 32-channel chunks per unit
+  static constexpr int TB = BITS == 4 ? 512 : 384;      // bytes per 32-row x 32-channel tile
+  static constexpr int UB = CH * TB;                    // code bytes per unit
+  static constexpr int SLOT = kSlotCodeBytes / 4 * BITS;
+  static constexpr int SU = SLOT / UB;                  // units per slot: 8, 4, 2
+  static constexpr int SCO = SLOT;                      // scales offset in a slot
+  static constexpr int ZO = SCO + SU * 64;              // zeros offset in a slot
   static constexpr int STRIDE = (ZO + SU * 16 + 127) / 128 * 128;
-  static constexpr int RING = kSlots * STRIDE;         // ring bytes per CTA
+  static constexpr int RING = kSlots * STRIDE;          // ring bytes per CTA
   static_assert(RING <= 160 * 1024, "rings too large for shared memory");
 };
 constexpr int kXsMaxBytes = 36 * 1024;  // x' of one pass staged in shared memory when it fits
@@ -134,15 +142,17 @@ __device__ __forceinline__ void warp_range(int cu0, int n, int w, int& wu0, int&
 // copy (with the barrier's expected byte count) and the scales + zeros copies can come from different lanes,
 // which proceed in parallel; the barrier's phase cannot complete before the arming arrival, so the order in
 // which the lanes' bytes land does not matter.
-template <int GS>
+template <int GS, int BITS>
 __device__ __forceinline__ void issue_codes(const GemvParams& p, int u, int c, uint8_t* slot, uint64_t* bar) {
-  mbar_arrive_expect_tx(bar, (unsigned)c * (unsigned)(Geo<GS>::UB + 80));
-  bulk_g2s(slot, p.qw + (size_t)u * Geo<GS>::UB, (unsigned)(c * Geo<GS>::UB), bar);
+  using Ge = Geo<GS, BITS>;
+  mbar_arrive_expect_tx(bar, (unsigned)c * (unsigned)(Ge::UB + 80));
+  bulk_g2s(slot, p.qw + (size_t)u * Ge::UB, (unsigned)(c * Ge::UB), bar);
 }
-template <int GS>
+template <int GS, int BITS>
 __device__ __forceinline__ void issue_meta(const GemvParams& p, int u, int c, uint8_t* slot, uint64_t* bar) {
-  bulk_g2s(slot + Geo<GS>::SCO, p.scales + (size_t)u * 32, (unsigned)(c * 64), bar);
-  bulk_g2s(slot + Geo<GS>::ZO, p.qzeros + (size_t)u * 4, (unsigned)(c * 16), bar);
+  using Ge = Geo<GS, BITS>;
+  bulk_g2s(slot + Ge::SCO, p.scales + (size_t)u * 32, (unsigned)(c * 64), bar);
+  bulk_g2s(slot + Ge::ZO, p.qzeros + (size_t)u * 4, (unsigned)(c * 16), bar);
 }
 
 // One unit: y rows (g + 8i, i = 0..3) x columns (8 nt + 2t + j) += S_row * sum_k (q - z) x'.
@@ -191,6 +201,76 @@ __device__ __forceinline__ void unit_mma(uint32_t codes, uint32_t scl, uint32_t 
         const uint32_t a1 = h2_as_u32(__hsub2(u32_as_h2(and_or<0x000F000Fu>(ub, m1024)), zlo[2 * h + 1]));
         const uint32_t a2 = h2_as_u32(__hsub2(u32_as_h2(and_or<0x00F000F0u>(ua, m64)), zhi[2 * h]));
         const uint32_t a3 = h2_as_u32(__hsub2(u32_as_h2(and_or<0x00F000F0u>(ub, m64)), zhi[2 * h + 1]));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma_16816_f32(c[nt][h][cc & 1], a0, a1, a2, a3, s ? xb[nt][cc].z : xb[nt][cc].x,
+                        s ? xb[nt][cc].w : xb[nt][cc].y);
+      }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      yacc[nt][2 * h][0] = fmaf(S[2 * h], c[nt][h][0][0] + c[nt][h][1][0], yacc[nt][2 * h][0]);
+      yacc[nt][2 * h][1] = fmaf(S[2 * h], c[nt][h][0][1] + c[nt][h][1][1], yacc[nt][2 * h][1]);
+      yacc[nt][2 * h + 1][0] = fmaf(S[2 * h + 1], c[nt][h][0][2] + c[nt][h][1][2], yacc[nt][2 * h + 1][0]);
+      yacc[nt][2 * h + 1][1] = fmaf(S[2 * h + 1], c[nt][h][0][3] + c[nt][h][1][3], yacc[nt][2 * h + 1][1]);
+    }
+}
+
+// The same unit for the packed 3-bit layout.  Lane (g, t) reads, for rows g and g + 8 of each half and each
+// chunk, the word holding the low 2-bit fields of its channel group t (word t / 2 of the row, the group's fields
+// at bit 8 (t % 2) on) and the row's high-bit word (word 2; pair p of group t at bits 4t + p and 4t + p + 16).
+// For each channel pair, (lo >> 2p) & 0x00030003 brought together with the high bits moved to bits 2 and 18 and
+// the exponent bits 0x6400 is the fp16 pair 1024 + q; one subtraction of (1024 + z) makes q - z exact, and the
+// MMA steps, B fragments and epilogue are those of the 4-bit unit.
+template <int NT, int CH>
+__device__ __forceinline__ void unit_mma3(uint32_t codes, uint32_t scl, uint32_t zer, int g, int t,
+                                          const uint4 (&xb)[NT][CH], float (&yacc)[NT][4][2]) {
+  uint32_t lo[2][2][CH], hl[2][2][CH], hh[2][2][CH];  // [half][row g / g + 8][chunk]
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int cc = 0; cc < CH; ++cc)
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const uint32_t row = codes + 384 * cc + 12 * (16 * h + g + 8 * rr);
+        lo[h][rr][cc] = ld_shared_u32(row + 4 * (t >> 1)) >> (8 * (t & 1));
+        const uint32_t w2 = ld_shared_u32(row + 8);
+        hl[h][rr][cc] = w2 << 2;  // the 64-bit value (w2 << 2), whose bits 4t + p + 2 and 4t + p + 18 ...
+        hh[h][rr][cc] = w2 >> 30;
+      }
+  const uint4 zw = ld_shared_v4(zer);
+  float S[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    S[i] = __half2float(__ushort_as_half(ld_shared_u16(scl + 2 * (g + 8 * i))));
+  const uint32_t zws[4] = {zw.x, zw.y, zw.z, zw.w};
+  __half2 z1024[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) z1024[i] = zero_1024((zws[i] >> (4 * g)) & 0xFu);
+  const uint32_t m1024 = magic_1024x2();
+  float c[NT][2][2][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) c[nt][h][pr][0] = c[nt][h][pr][1] = c[nt][h][pr][2] = c[nt][h][pr][3] = 0.f;
+  // fp16 pair (1024 + q) of channel pair p of this lane's group, for one row
+  auto pair = [&](int h, int rr, int cc, int p) -> uint32_t {
+    const uint32_t hb = __funnelshift_r(hl[h][rr][cc], hh[h][rr][cc], 4 * t + p);  // ... land at bits 2 and 18
+    return and_or<0x00030003u>(lo[h][rr][cc] >> (2 * p), and_or<0x00040004u>(hb, m1024));
+  };
+#pragma unroll
+  for (int cc = 0; cc < CH; ++cc)
+#pragma unroll
+    for (int s = 0; s < 2; ++s)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t a0 = h2_as_u32(__hsub2(u32_as_h2(pair(h, 0, cc, 2 * s)), z1024[2 * h]));
+        const uint32_t a1 = h2_as_u32(__hsub2(u32_as_h2(pair(h, 1, cc, 2 * s)), z1024[2 * h + 1]));
+        const uint32_t a2 = h2_as_u32(__hsub2(u32_as_h2(pair(h, 0, cc, 2 * s + 1)), z1024[2 * h]));
+        const uint32_t a3 = h2_as_u32(__hsub2(u32_as_h2(pair(h, 1, cc, 2 * s + 1)), z1024[2 * h + 1]));
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
           mma_16816_f32(c[nt][h][cc & 1], a0, a1, a2, a3, s ? xb[nt][cc].z : xb[nt][cc].x,
@@ -329,10 +409,10 @@ __host__ __device__ constexpr int gemv_xs_bytes(int rows, int xpitch) { return (
 // (before any dependency wait), later ones when the consumer has released the slot.
 constexpr int kSlotLanes = kSlots <= 16 ? kSlots : 32;  // lanes that issue codes; kSlots <= 16: one more lane for meta
 static_assert(kSlots <= 32, "one producer warp serves at most 32 slots");
-template <int GS>
+template <int GS, int BITS>
 __device__ __forceinline__ void gemv_producer(const GemvParams& p, uint8_t* ring, uint64_t* full, uint64_t* empty,
                                               int cu0, int n, int lane) {
-  constexpr int kSU = Geo<GS>::SU;
+  constexpr int kSU = Geo<GS, BITS>::SU;
   const bool split = kSlots <= 16;
   const int j = split ? lane % 16 : lane;
   const bool does_codes = lane < kSlotLanes, does_meta = split ? (lane >= 16 && j < kSlots) : does_codes;
@@ -340,11 +420,11 @@ __device__ __forceinline__ void gemv_producer(const GemvParams& p, uint8_t* ring
   int wu0, nw;
   warp_range(cu0, n, j / kRing, wu0, nw);
   const int si = j % kRing;
-  uint8_t* slot = ring + (size_t)j * Geo<GS>::STRIDE;
+  uint8_t* slot = ring + (size_t)j * Geo<GS, BITS>::STRIDE;
   auto issue = [&](int sq) {
     const int u = wu0 + sq * kSU, c = min(kSU, nw - sq * kSU);
-    if (does_codes) issue_codes<GS>(p, u, c, slot, &full[j]);
-    if (does_meta) issue_meta<GS>(p, u, c, slot, &full[j]);
+    if (does_codes) issue_codes<GS, BITS>(p, u, c, slot, &full[j]);
+    if (does_meta) issue_meta<GS, BITS>(p, u, c, slot, &full[j]);
   };
   int next = si;  // next slot sequence number to issue
   if (next * kSU < nw) {
@@ -369,9 +449,9 @@ __device__ __forceinline__ void gemv_producer(const GemvParams& p, uint8_t* ring
   }
 }
 
-template <int NT, bool XS, bool DIVS, int GS>
+template <int NT, bool XS, bool DIVS, int GS, int BITS>
 __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
-  using Ge = Geo<GS>;
+  using Ge = Geo<GS, BITS>;
   constexpr int kSU = Ge::SU, CH = Ge::CH;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[kSlots];
@@ -403,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
       for (unsigned long long o = a; o < e; o += 32768ull)
         prefetch_l2_bulk(p.pf + o, (unsigned)(e - o < 32768ull ? e - o : 32768ull));
     }
-    gemv_producer<GS>(p, ring, full, empty, cu0, n, lane);
+    gemv_producer<GS, BITS>(p, ring, full, empty, cu0, n, lane);
     return;
   }
 
@@ -505,8 +585,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
         ok = __all_sync(0xFFFFFFFFu, mbar_wait_backoff(&full[warp * kRing + si], (unsigned)(sq / kRing) & 1u, p.status));
         if (!ok) break;  // warp-uniform
       }
-      unit_mma<NT, CH>(slot + (uint32_t)(ui * Ge::UB), slot + (uint32_t)(Ge::SCO + ui * 64),
-                       slot + (uint32_t)(Ge::ZO + ui * 16), g4, t4, xcur, yacc);
+      if (BITS == 4)
+        unit_mma<NT, CH>(slot + (uint32_t)(ui * Ge::UB), slot + (uint32_t)(Ge::SCO + ui * 64),
+                         slot + (uint32_t)(Ge::ZO + ui * 16), g4, t4, xcur, yacc);
+      else
+        unit_mma3<NT, CH>(slot + (uint32_t)(ui * Ge::UB), slot + (uint32_t)(Ge::SCO + ui * 64),
+                          slot + (uint32_t)(Ge::ZO + ui * 16), g4, t4, xcur, yacc);
       if (ui == kSU - 1 || t == nw - 1) {  // last unit of the slot: every lane has read it; release it
         __syncwarp();
         if (lane == 0) mbar_arrive_addr(empty_addr + 8u * (uint32_t)si);
@@ -564,13 +648,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const GemvParams p) {
 
 namespace {
 
-template <int NT, bool XS, bool DIVS, int GS>
+template <int NT, bool XS, bool DIVS, int GS, int BITS>
 bool gemv_smem_attr() {
   static bool done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(gemv_kernel<NT, XS, DIVS, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gemv_kernel<NT, XS, DIVS, GS, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kMaxDynSmem) != cudaSuccess)
       return false;
     done[dev] = true;
@@ -578,7 +662,8 @@ bool gemv_smem_attr() {
   return true;
 }
 
-int ring_bytes(int gs) {
+int ring_bytes(int gs, int bits) {
+  if (bits == 3) return gs == 64 ? Geo<64, 3>::RING : gs == 128 ? Geo<128, 3>::RING : Geo<256, 3>::RING;
   return gs == 64 ? Geo<64>::RING : gs == 128 ? Geo<128>::RING : Geo<256>::RING;
 }
 
@@ -595,7 +680,7 @@ struct GemvPlan {
 //  - more row blocks, evenly enough divisible: each CTA takes a balanced run of whole row blocks;
 //  - otherwise (a few row blocks more than CTAs) the units are spread evenly over the CTAs and the row
 //    blocks cut by CTA boundaries are combined in the workspace.
-GemvPlan plan_gemv(int M, int N, int K, int gs, bool divide = false) {
+GemvPlan plan_gemv(int M, int N, int K, int gs, bool divide = false, int bits = 4) {
   GemvPlan pl{};
   pl.NT = M <= 8 ? 1 : 2;
   pl.mts = M < 8 * pl.NT ? M : 8 * pl.NT;
@@ -629,22 +714,28 @@ GemvPlan plan_gemv(int M, int N, int K, int gs, bool divide = false) {
   // The fused 1/s variant divides the staged copy, so it stages whatever fits beside the rings and partials.
   const int units_per_warp = pl.U / pl.P / kNW;
   pl.xs = (divide || (pl.mts * pl.xpitch * 2 <= kXsMaxBytes && 3 * units_per_warp >= pl.G)) &&
-          ring_bytes(gs) + gemv_xs_bytes(pl.mts, pl.xpitch) + gemv_part_bytes(pl.mts) <= kMaxDynSmem;
+          ring_bytes(gs, bits) + gemv_xs_bytes(pl.mts, pl.xpitch) + gemv_part_bytes(pl.mts) <= kMaxDynSmem;
   return pl;
 }
 
-template <int NT, bool XS, bool DIVS, int GS>
+template <int NT, bool XS, bool DIVS, int GS, int BITS>
 cudaError_t launch_nt(const GemvParams& p, int mcount, cudaStream_t st) {
-  if (!gemv_smem_attr<NT, XS, DIVS, GS>()) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)Geo<GS>::RING + (XS ? gemv_xs_bytes(mcount, p.xpitch) : 0) + gemv_part_bytes(mcount);
-  return launch_pdl(gemv_kernel<NT, XS, DIVS, GS>, dim3((unsigned)p.P), dim3(kThreads), smem, st, p);
+  if (!gemv_smem_attr<NT, XS, DIVS, GS, BITS>()) return cudaErrorInvalidValue;
+  const size_t smem =
+      (size_t)Geo<GS, BITS>::RING + (XS ? gemv_xs_bytes(mcount, p.xpitch) : 0) + gemv_part_bytes(mcount);
+  return launch_pdl(gemv_kernel<NT, XS, DIVS, GS, BITS>, dim3((unsigned)p.P), dim3(kThreads), smem, st, p);
 }
 
 template <int GS>
-cudaError_t launch_gs(const GemvParams& p, int NT, bool xs, bool divide, int mcount, cudaStream_t st) {
-  if (divide) return NT == 1 ? launch_nt<1, true, true, GS>(p, mcount, st) : launch_nt<2, true, true, GS>(p, mcount, st);
-  if (NT == 1) return xs ? launch_nt<1, true, false, GS>(p, mcount, st) : launch_nt<1, false, false, GS>(p, mcount, st);
-  return xs ? launch_nt<2, true, false, GS>(p, mcount, st) : launch_nt<2, false, false, GS>(p, mcount, st);
+cudaError_t launch_gs(const GemvParams& p, int NT, bool xs, bool divide, int mcount, cudaStream_t st, int bits) {
+  if (bits == 3) {  // the 3-bit layout: plain x' only
+    if (NT == 1) return xs ? launch_nt<1, true, false, GS, 3>(p, mcount, st) : launch_nt<1, false, false, GS, 3>(p, mcount, st);
+    return xs ? launch_nt<2, true, false, GS, 3>(p, mcount, st) : launch_nt<2, false, false, GS, 3>(p, mcount, st);
+  }
+  if (divide)
+    return NT == 1 ? launch_nt<1, true, true, GS, 4>(p, mcount, st) : launch_nt<2, true, true, GS, 4>(p, mcount, st);
+  if (NT == 1) return xs ? launch_nt<1, true, false, GS, 4>(p, mcount, st) : launch_nt<1, false, false, GS, 4>(p, mcount, st);
+  return xs ? launch_nt<2, true, false, GS, 4>(p, mcount, st) : launch_nt<2, false, false, GS, 4>(p, mcount, st);
 }
 
 }  // namespace
@@ -656,7 +747,8 @@ size_t gemv_workspace_bytes(int M, int N, int K, int g) {
 
 awq_status gemv_launch(const LinearArgs& a) {
   const bool divide = a.inv_s != nullptr;
-  const GemvPlan pl = plan_gemv(a.M, a.N, a.K, a.g, divide);
+  if (a.bits == 3 && (divide || a.epi)) return AWQ_ERR_UNSUPPORTED;
+  const GemvPlan pl = plan_gemv(a.M, a.N, a.K, a.g, divide, a.bits);
   if (divide && !pl.xs) return AWQ_ERR_UNSUPPORTED;  // x / s needs the staged copy
   if ((size_t)pl.RB * 4 > kWorkspaceCounterBytes) return AWQ_ERR_UNSUPPORTED;
   if (pl.part_bytes > 0 && (a.ws == nullptr || a.ws_bytes < kWorkspaceCounterBytes + pl.part_bytes))
@@ -696,9 +788,9 @@ awq_status gemv_launch(const LinearArgs& a) {
     const int mcount = a.M - m0 < rows ? a.M - m0 : rows;
     cudaError_t e;
     switch (a.g) {
-      case 64: e = launch_gs<64>(p, pl.NT, pl.xs, divide, mcount, a.st); break;
-      case 256: e = launch_gs<256>(p, pl.NT, pl.xs, divide, mcount, a.st); break;
-      default: e = launch_gs<128>(p, pl.NT, pl.xs, divide, mcount, a.st); break;
+      case 64: e = launch_gs<64>(p, pl.NT, pl.xs, divide, mcount, a.st, a.bits); break;
+      case 256: e = launch_gs<256>(p, pl.NT, pl.xs, divide, mcount, a.st, a.bits); break;
+      default: e = launch_gs<128>(p, pl.NT, pl.xs, divide, mcount, a.st, a.bits); break;
     }
     if (e != cudaSuccess) return AWQ_ERR_CUDA;
   }

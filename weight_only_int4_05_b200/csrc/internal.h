@@ -46,7 +46,7 @@ awq_status prep_inv_scale_launch(const uint16_t* x, const uint16_t* s, int M, in
 // (gate|up, N = 2 * NI, NI % 16 == 0): row 32j + i of the packed weight is W[16j + i] for i < 16 and
 // W2[16j + i - 16] for i >= 16.
 awq_status pack_launch(const uint16_t* W, const uint16_t* W2, const uint16_t* s, int N, int K, int g, uint32_t* qw,
-                       uint16_t* scales, uint32_t* qz, cudaStream_t st, int w_bit = 4);
+                       uint16_t* scales, uint32_t* qz, cudaStream_t st, int w_bit = 4, int storage_bits = 4);
 
 // One linear-layer call as the kernels see it.
 struct LinearArgs {
@@ -57,6 +57,7 @@ struct LinearArgs {
   uint16_t* y = nullptr;
   int M = 0, N = 0, K = 0, g = 128;
   int epi = 0;  // 0: y [M][N]; 1: gate|up packed by pack_launch with W2, y [M][N/2] = silu(gate) * up
+  int bits = 4;  // code layout: 4 (the 4-bit layout) or 3 (the packed 3-bit layout; GEMV only, no epi / inv_s)
   void* ws = nullptr;
   size_t ws_bytes = 0;
   unsigned* status = nullptr;
