@@ -202,15 +202,18 @@ class DecodeStack:
     """32 layers x 7 packed linears, inputs x' and outputs y resident in HBM, one CUDA graph per step."""
 
     def __init__(self, device, seed=0, M=1, layers=LAYERS, inputs_fn=None, prefetch=False, fused=False,
-                 inv_s_fused=False, silu=False):
+                 inv_s_fused=False, silu=False, inv_s_two_pass=False):
         """inputs_fn(layer, linear, M, N, K) -> (W, xcal, x) fp16 device tensors; default: the seeded
         device generator of the synthetic workload.  prefetch: each call passes the next linear's packed
         weight as an L2 prefetch hint (w4a16_linear_pf).  fused: 4 linears per layer (FUSED_SHAPES).
         inv_s_fused: the resident activations are the raw x and every call is w4a16_gemv_s(x, s), which
         divides by the AWQ scale inside the kernel (no separate 1/s pass).  silu (with fused): the gate|up
         linear is packed by awq_pack_gate_up and called as w4a16_gate_up_silu, writing silu(gate) * up
-        (14336 columns) instead of both projections."""
+        (14336 columns) instead of both projections.  inv_s_two_pass: the same raw activations, but every linear
+        is the two launches awq_apply_inv_scale(x, s) then w4a16_linear (the unfused form of inv_s_fused)."""
         self.prefetch = prefetch
+        self.two_pass = inv_s_two_pass
+        inv_s_fused = inv_s_fused or inv_s_two_pass
         self.silu = silu and fused
         self.inv_s_fused = inv_s_fused
         layer_shapes = FUSED_SHAPES if fused else DECODE_SHAPES
@@ -222,6 +225,7 @@ class DecodeStack:
         self.W4, self.torch, self.device, self.M = W4, torch, device, M
         self.entries = []  # (packed weight, x' view, y view)
         self.s_list = []   # AWQ scales (inv_s_fused only)
+        self.xp_list = []  # scaled activations formed every step (inv_s_two_pass only)
         shapes = [(li, name, K, N) for li in range(layers) for (name, K, N) in layer_shapes]
         self.h2d_elems = sum(M * K for _, _, K, _ in shapes)
         self.d2h_elems = sum(M * N for _, _, _, N in shapes)
@@ -250,10 +254,14 @@ class DecodeStack:
             if gate_up:
                 yv = yv.reshape(-1)[:M * N // 2].view(M, N // 2)
             self.entries.append((pw, xv, yv, K, N))
+            if self.two_pass:
+                self.xp_list.append(torch.empty_like(xv))
             xo += M * K
             yo += M * N
             del Wt, xcal, x
         self.launches_per_step = sum(self._launches(K, N) for _, _, _, K, N in self.entries)
+        if self.two_pass:
+            self.launches_per_step += len(self.entries)  # one inv_scale_kernel per linear
         need = max(W4.w4a16_workspace_bytes(W4.MODE_LINEAR, M, N, K) for _, _, _, K, N in self.entries)
         W4.reserve_workspace(need, device)
         torch.cuda.synchronize(device)
@@ -268,7 +276,10 @@ class DecodeStack:
     def eager_step(self):
         n = len(self.entries)
         for i, (pw, xv, yv, _, _) in enumerate(self.entries):
-            if self.inv_s_fused:
+            if self.two_pass:
+                self.W4.awq_apply_inv_scale(xv, self.s_list[i], out=self.xp_list[i])
+                self.W4.w4a16_linear(self.xp_list[i], pw, out=yv)
+            elif self.inv_s_fused:
                 self.W4.w4a16_gemv_s(xv, self.s_list[i], pw, out=yv)
             elif yv.shape[1] * 2 == pw.N and self.silu:
                 self.W4.w4a16_gate_up_silu(xv, pw, out=yv)
@@ -845,6 +856,19 @@ def run_gpu(args):
     del sstack
     torch.cuda.empty_cache()
 
+    # ---- the same work unfused: awq_apply_inv_scale then w4a16_linear for every linear (448 launches per token)
+    tstack = DecodeStack(device, inv_s_two_pass=True)
+    tstack.capture()
+    t_s, t_clocks = time_steps(tstack.step, args.steps, args.warmup, device, ClockSampler(gpu_uuid_id(device)))
+    t_value = aggregate_value(s_bytes, args.steps, world, t_s)
+    decode_inv_s_two_pass = {"value": t_value, "unit": "GB/s", "ms_per_step": t_s / args.steps * 1e3,
+                             "frac": t_value / world / peaks["hbm_gbs"], "steps": args.steps, "clocks": t_clocks,
+                             "bytes_per_step": s_bytes, "gpu_launches": tstack.launches_per_step * args.steps,
+                             "workload": "the same raw activations, unfused: awq_apply_inv_scale then w4a16_linear "
+                                         "for every linear (the same algorithmic bytes as decode_inv_s_fused)"}
+    del tstack
+    torch.cuda.empty_cache()
+
     # ---- head 2: prefill GEMM at M=2048, timed over at least 150 ms
     pre = PrefillGemm(device)
     pre.capture()
@@ -898,6 +922,7 @@ def run_gpu(args):
                     "steps": e2e_steps},
             "gemm": gemm, "decode_sweep": sweep, "tiny": tiny, "pack": pack, "crossover": crossover,
             "decode_prefetch_hint": decode_pf, "decode_fused": decode_fused, "decode_inv_s_fused": decode_inv_s,
+            "decode_inv_s_two_pass": decode_inv_s_two_pass,
             "decode_fused_silu": decode_fused_silu, "group_sizes": groups, "int3_layout": int3, "awq_search": search,
             "gptq": gptq}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
