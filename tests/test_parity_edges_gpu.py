@@ -242,3 +242,27 @@ def test_prefill_gemm_m2048_every_tile_quarter_and_chunk():
                     ms.append(tt * 256 + ch * 16 + int(rng.integers(0, 16)))
     ms, ns = np.array(ms, np.int32), np.array(ns, np.int32)
     assert_within_tolerance(y[ms, ns], case.y_pairs(ms, ns), "gemm M=2048 every tile")
+
+
+def test_prefill_gemm_short_last_wave_split():
+    """(K, N) = (4096, 14336) at M = 2048 is 896 output tiles: six whole waves on 148 SMs run as one launch and
+    the last 8 tiles as a second launch with K split 8 ways (workspace partials summed in split order).  One
+    sample in every (32-row quarter, 16-column chunk) of those 8 tiles and of 8 tiles of the first launch."""
+    M, K, N = 2048, 4096, 14336
+    case = OracleCase(0, 3, 2, 5, M, N, K)
+    s = W4.awq_act_scale(dev(case.xcal))
+    xp = W4.awq_apply_inv_scale(dev(case.x), s)
+    pw = W4.awq_pack(dev(case.W), s)
+    y = W4.w4a16_gemm(xp, pw).float().cpu().numpy()
+    n_tiles = N // 128
+    rng = np.random.default_rng(13)
+    ms, ns = [], []
+    for tile in list(range(888, 896)) + list(range(880, 888)):
+        nt, tt = tile % n_tiles, tile // n_tiles
+        for qq in range(4):
+            for ch in range(16):
+                ns.append(nt * 128 + qq * 32 + int(rng.integers(0, 32)))
+                ms.append(tt * 256 + ch * 16 + int(rng.integers(0, 16)))
+    ms, ns = np.array(ms, np.int32), np.array(ns, np.int32)
+    assert_within_tolerance(y[ms, ns], case.y_pairs(ms, ns), "gemm M=2048 last-wave split")
+    assert W4.awq_last_device_status() == 0

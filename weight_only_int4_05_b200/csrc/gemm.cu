@@ -54,6 +54,7 @@ struct GemmParams {
   unsigned* ws_cnt;  // per-tile arrival counters (zero between calls)
   int M, N, Np, K, KB, BT, ST, tmem_cols;
   int splits, kb_per_split;  // k-blocks [split * kb_per_split, ...) per CTA
+  int tile_base, n_tiles;    // CTA x handles output tile tile_base + x (n-tile = tile % n_tiles, t-tile = tile / n_tiles)
   uint32_t idesc;
 };
 
@@ -224,7 +225,7 @@ __device__ __forceinline__ void gemm_dequant_epilogue(const GemmParams& p, uint8
     return;
   }
   // ---- split-K: fp32 partial tile to the workspace; the last split to arrive sums them in order
-  const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+  const int tile = blockIdx.x;  // this launch's tile slot in the workspace and the counters
   float* tile_ws = p.ws_part + (size_t)tile * p.splits * p.BT * 128;
   float* mine = tile_ws + (size_t)blockIdx.z * p.BT * 128;  // [column][row]
   if (!aborted) {  // an aborted CTA has no valid accumulator, but still arrives on the tile counter below
@@ -276,7 +277,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kBN, t0 = blockIdx.y * p.BT;
+  const int tile = p.tile_base + (int)blockIdx.x;
+  const int n0 = (tile % p.n_tiles) * kBN, t0 = (tile / p.n_tiles) * p.BT;
   const int rb_avail = min(4, (p.Np - n0) / 32);
   const int kb0 = blockIdx.z * p.kb_per_split;
   const int nkb = min(p.kb_per_split, p.KB - kb0);
@@ -369,11 +371,15 @@ bool smem_attr_set(int smem) {
 
 struct GemmPlan {
   int BT, n_tiles, t_tiles, KB, splits, kb_per_split;
+  int main_tiles;                        // tiles of the first launch (all of them unless there is a tail)
+  int tail_tiles, tail_splits, tail_kbs;  // a short last wave, run as a second launch with K split
   size_t part_bytes;
 };
 
-// Split K when the output tiles alone cannot occupy the SMs: as many splits as fit in one wave, each
-// with at least 4 k-blocks.
+// Split K when the output tiles alone cannot occupy the SMs: as many splits as fit in one wave, each with at
+// least 4 k-blocks.  When the tiles fill the SMs but leave a short last wave (at most a quarter of the SMs,
+// e.g. 896 tiles = 6 waves + 8), the whole waves run as one launch and the last few tiles as a second
+// launch with K split over the SMs, so the last wave takes a fraction of a tile's time instead of a whole one.
 GemmPlan plan_gemm(int M, int N, int K) {  // the same plan for every group size
   GemmPlan g{};
   g.BT = pick_bt(M);
@@ -381,13 +387,35 @@ GemmPlan plan_gemm(int M, int N, int K) {  // the same plan for every group size
   g.t_tiles = (M + g.BT - 1) / g.BT;
   g.KB = K / kBK;
   const int tiles = g.n_tiles * g.t_tiles;
-  int s = tiles >= num_sms() ? 1 : num_sms() / tiles;
+  const int sms = num_sms();
   const int max_by_k = g.KB / 4 > 0 ? g.KB / 4 : 1;
-  if (s > max_by_k) s = max_by_k;
-  if (s < 1) s = 1;
-  g.kb_per_split = (g.KB + s - 1) / s;
-  g.splits = (g.KB + g.kb_per_split - 1) / g.kb_per_split;  // no empty split
-  g.part_bytes = g.splits > 1 ? (size_t)tiles * g.splits * g.BT * 128 * sizeof(float) : 0;
+  auto split_for = [&](int count, int& splits, int& kbs) {
+    int s = count >= sms ? 1 : sms / count;
+    if (s > max_by_k) s = max_by_k;
+    if (s < 1) s = 1;
+    kbs = (g.KB + s - 1) / s;
+    splits = (g.KB + kbs - 1) / kbs;  // no empty split
+  };
+#ifndef AWQ_GEMM_TAIL_SPLITS  // cap on the splits of the last-wave launch (measured on 4096 -> 14336 at M = 2048:
+#define AWQ_GEMM_TAIL_SPLITS 8  // 292.6 us as one launch, 280.6 / 282.1 / 278.6 us with 2 / 4 / 8 splits)
+#endif
+  const int tail = tiles > sms ? tiles % sms : 0;
+  if (AWQ_GEMM_TAIL_SPLITS > 1 && tail > 0 && tail * 4 <= sms) {
+    g.main_tiles = tiles - tail;
+    g.splits = 1;
+    g.kb_per_split = g.KB;
+    g.tail_tiles = tail;
+    split_for(tail, g.tail_splits, g.tail_kbs);
+    if (g.tail_splits > AWQ_GEMM_TAIL_SPLITS) {  // fewer, longer splits: the last arriver sums fewer partials
+      g.tail_kbs = (g.KB + AWQ_GEMM_TAIL_SPLITS - 1) / AWQ_GEMM_TAIL_SPLITS;
+      g.tail_splits = (g.KB + g.tail_kbs - 1) / g.tail_kbs;
+    }
+    g.part_bytes = g.tail_splits > 1 ? (size_t)tail * g.tail_splits * g.BT * 128 * sizeof(float) : 0;
+  } else {
+    g.main_tiles = tiles;
+    split_for(tiles, g.splits, g.kb_per_split);
+    g.part_bytes = g.splits > 1 ? (size_t)tiles * g.splits * g.BT * 128 * sizeof(float) : 0;
+  }
   return g;
 }
 
@@ -428,6 +456,8 @@ awq_status gemm_launch(const LinearArgs& a) {
   p.ws_part = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWorkspaceCounterBytes) : nullptr;
   p.splits = g.splits;
   p.kb_per_split = g.kb_per_split;
+  p.tile_base = 0;
+  p.n_tiles = g.n_tiles;
   p.BT = g.BT;
   const int sb = stage_bytes(p.BT);
   p.ST = (kMaxSmem - 2048) / sb;
@@ -476,8 +506,15 @@ awq_status gemm_launch(const LinearArgs& a) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return AWQ_ERR_CUDA;
   }
-  const dim3 grid((unsigned)g.n_tiles, (unsigned)g.t_tiles, (unsigned)g.splits);
-  cudaError_t e = launch_pdl(gemm_kernel, grid, dim3(kGemmThreads), (size_t)smem, a.st, maps, p);
+  cudaError_t e = launch_pdl(gemm_kernel, dim3((unsigned)g.main_tiles, 1u, (unsigned)g.splits), dim3(kGemmThreads),
+                             (size_t)smem, a.st, maps, p);
+  if (e == cudaSuccess && g.tail_tiles > 0) {  // the short last wave, K split over the SMs
+    p.tile_base = g.main_tiles;
+    p.splits = g.tail_splits;
+    p.kb_per_split = g.tail_kbs;
+    e = launch_pdl(gemm_kernel, dim3((unsigned)g.tail_tiles, 1u, (unsigned)g.tail_splits), dim3(kGemmThreads),
+                   (size_t)smem, a.st, maps, p);
+  }
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
