@@ -28,6 +28,7 @@ __all__ = [
     "w4a16_gemv", "w4a16_gemm", "w4a16_linear", "w4a16_gemv_max_m", "w4a16_workspace_bytes",
     "awq_last_device_status", "reserve_workspace", "lib_path", "w4a16_gemv_noalloc",
     "awq_selftest_wait_timeout", "w4a16_linear_pf", "w4a16_gemv_s", "awq_pack_gate_up", "w4a16_gate_up_silu",
+    "SearchResult", "awq_search_scale", "gptq_quantize", "awq_pack3", "w3a16_gemv",
 ]
 
 
