@@ -11,8 +11,8 @@
 //
 // Warp roles.  One producer warp per CTA fills every slot with TMA bulk copies -- the codes, scales and zeros
 // of the 8 KB of consecutive units a slot holds, three copies completing on the slot's "full" mbarrier -- and
-// refills a slot when
-// its consumer has released it on the slot's "empty" mbarrier.  Slot j of the CTA (warp j / kRing, ring index j % kRing) is
+// refills a slot when its consumer has released it on the slot's "empty" mbarrier (the first fill of a warp's
+// second slot is held back a little; see gemv_producer).  Slot j of the CTA (warp j / kRing, ring index j % kRing) is
 // served by producer lane j % 32: a thread completes about one bulk copy per ~770 cycles whatever its size,
 // and a copy waiting behind another one stalls its thread, so spreading the slots over the lanes keeps the
 // copies in parallel and keeps every issue stall off the consumer warps.
@@ -405,10 +405,29 @@ __host__ __device__ constexpr int gemv_xs_bytes(int rows, int xpitch) { return (
 // lanes below kSlotLanes issue the slot's codes copy (and arm its barrier), lanes from kSlotLanes on issue its
 // scales and zeros when there are enough lanes, so the big and small copies of a slot are serviced in
 // parallel.  The warp's slot sequence number sq = 0, 1, ... covers its units [sq * kSU, sq * kSU + kSU) (kSU
-// units per slot); ring index si takes the sequence numbers si, si + kRing, ...  The first use of each slot is issued at once
-// (before any dependency wait), later ones when the consumer has released the slot.
+// units per slot); ring index si takes the sequence numbers si, si + kRing, ...  The first fill of ring index 0
+// is issued at once (before any dependency wait), the first fill of ring index si > 0 after si * kStaggerCycles
+// cycles, and every later fill when the consumer has released the slot.
+//
+// Why the stagger: at a kernel's start every CTA asks for all its slots at once (about 20 MB over the GPU), and
+// DRAM serves the outstanding copies side by side, so the slot each warp needs first lands only near the end of
+// the whole burst.  Holding back the second slots lets the first ones land sooner.  Measured on one B200 (µs
+// per call at M = 1, programmatic dependent launch between calls): the 224-linear decode stack 1621 -> 1589 per
+// token, 14336 -> 4096 10.83 -> 10.34, 4096 -> 14336 10.66 -> 10.86, q/o and k/v unchanged.  Issuing the second
+// slot as soon as the first has landed instead was slower on the single linears (14336 -> 4096 11.42).
 constexpr int kSlotLanes = kSlots <= 16 ? kSlots : 32;  // lanes that issue codes; kSlots <= 16: one more lane for meta
 static_assert(kSlots <= 32, "one producer warp serves at most 32 slots");
+#ifndef AWQ_GEMV_STAGGER_CYCLES
+#define AWQ_GEMV_STAGGER_CYCLES 4000  // about 2 us at the 1965 MHz boost clock
+#endif
+constexpr long long kStaggerCycles = AWQ_GEMV_STAGGER_CYCLES;
+
+// Bounded pause of the calling thread (SM clock cycles).
+__device__ __forceinline__ void pause_cycles(long long cycles) {
+  const long long c0 = clock64();
+  while (clock64() - c0 < cycles) __nanosleep(32);
+}
+
 template <int GS, int BITS>
 __device__ __forceinline__ void gemv_producer(const GemvParams& p, uint8_t* ring, uint64_t* full, uint64_t* empty,
                                               int cu0, int n, int lane) {
@@ -428,6 +447,7 @@ __device__ __forceinline__ void gemv_producer(const GemvParams& p, uint8_t* ring
   };
   int next = si;  // next slot sequence number to issue
   if (next * kSU < nw) {
+    if (si > 0 && kStaggerCycles > 0) pause_cycles(kStaggerCycles * si);
     issue(next);
     next += kRing;
   }
