@@ -462,6 +462,14 @@ awq_status gemm_launch(const LinearArgs& a) {
   const int sb = stage_bytes(p.BT);
   p.ST = (kMaxSmem - 2048) / sb;
   if (p.ST > 8) p.ST = 8;
+  // The dequant warpgroups take k-blocks round robin (kb % kDequantWG) and stage s = kb % ST.  With ST a
+  // multiple of kDequantWG every stage always belongs to the same warpgroup, which then waits for the stage's
+  // phases strictly in order.  Otherwise two warpgroups alternate on a stage, and when copies land out of
+  // order one of them can reach phase P + 2 of full[s] while P + 1 is still in flight: its parity wait then
+  // matches phase P and it reads a stage that is still being filled (and its early arrival shifts afull[s]
+  // one phase ahead of the MMA thread, which then waits until its bounded wait gives up).
+  p.ST = p.ST / kDequantWG * kDequantWG;
+  if (p.ST < kDequantWG) return AWQ_ERR_UNSUPPORTED;
   p.tmem_cols = pow2_at_least(p.BT, 32);
   p.idesc = umma_idesc_f16(kBN, p.BT);
   const int smem = p.ST * sb + 1024 + 256;
